@@ -1,0 +1,274 @@
+/*
+ * Plain fp64 CPU oracle for paged MLA latent-attention decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this file.  It shares no code,
+ * header, table or helper with the CUDA library, and the library never calls
+ * it.
+ *
+ * What it computes (one query row = one (sequence b, query token t, head h)):
+ *
+ *   n      = number of cached positions the row may see
+ *   kv_j   = dequantised 576-value row of position j, looked up through the
+ *            page table: page = page_table[b][j / 16], slot = j % 16
+ *   s_j    = sm_scale * ( q_lat . kv_j[0:512] + q_pe . kv_j[512:576] )
+ *   M      = max_j s_j,   Z = sum_j exp(s_j - M),   lse = M + ln Z
+ *   out[d] = sum_j exp(s_j - M) / Z * kv_j[d]          for d < 512
+ *
+ * Sources: the compressed KV history of 576 values per position and its
+ * per-position byte count ("Inside Kimi K3 optimisation work", section 1,
+ * DCP paragraph); 16-token pages ("Kimi K2.6 DFlash on 8x MI300X", hardware
+ * stack, BLOCK_SIZE=16); every query head attends to the cached positions on
+ * its own ("Inside Kimi K3 optimisation work", section 4, head padding);
+ * partial answers carry normalisation information and merge exactly
+ * (section 1, DCP; section 4, history split).  The 512 + 64 split of the 576
+ * values, the value = latent reading and the per-token FP8 scale are the
+ * plainest reading of the problem statement: the pages give only the
+ * 576-value total and a dynamically computed FP8 scale.
+ *
+ * Visibility: without an explicit per-token count, query token t of a
+ * sequence with ctx cached positions sits at position ctx - T + t (the last T
+ * cached positions are the query tokens themselves) and sees every position
+ * up to and including itself: n = ctx - T + t + 1.
+ *
+ * An empty visible set gives out = 0 and lse = -inf.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define ORACLE_PAGE 16
+#define ORACLE_DL 512
+#define ORACLE_DR 64
+#define ORACLE_D (ORACLE_DL + ORACLE_DR)
+
+enum { ORACLE_KV_BF16 = 0, ORACLE_KV_FP8 = 1 };
+
+/* bfloat16 is the upper half of an IEEE binary32; widening is exact. */
+double oracle_bf16_to_f64(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* FP8 e4m3fn from its format definition: 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent 0 is subnormal (m/8 * 2^-6); the single
+ * pattern S.1111.111 is NaN; there is no infinity; largest finite is 448. */
+double oracle_e4m3_to_f64(uint8_t byte) {
+    int sign = byte >> 7;
+    int e = (byte >> 3) & 0xF;
+    int m = byte & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+typedef struct {
+    int B, T, H;
+    const uint16_t *q_lat;   /* [B,T,H,512] bf16 bits */
+    const uint16_t *q_pe;    /* [B,T,H,64]  bf16 bits */
+    const void *kv_pages;    /* [P,16,576] bf16 bits or e4m3fn bytes */
+    int kv_dtype;
+    const float *kv_scale;   /* [P,16] for FP8, else NULL */
+    int num_pages;
+    const int32_t *page_table;
+    int page_table_stride;
+    const int32_t *ctx_lens; /* [B] */
+    const int32_t *vis_lens; /* [B,T] or NULL */
+    double sm_scale;
+} oracle_problem;
+
+/* One dequantised KV value: element d of the row stored at (page, slot). */
+static double kv_value(const oracle_problem *p, int64_t page, int slot, int d) {
+    int64_t row = page * ORACLE_PAGE + slot;
+    if (p->kv_dtype == ORACLE_KV_BF16) {
+        const uint16_t *kv = (const uint16_t *)p->kv_pages;
+        return oracle_bf16_to_f64(kv[row * ORACLE_D + d]);
+    } else {
+        const uint8_t *kv = (const uint8_t *)p->kv_pages;
+        return oracle_e4m3_to_f64(kv[row * ORACLE_D + d]) * (double)p->kv_scale[row];
+    }
+}
+
+static int visible_count(const oracle_problem *p, int b, int t) {
+    if (p->vis_lens) return p->vis_lens[(int64_t)b * p->T + t];
+    return p->ctx_lens[b] - p->T + t + 1;
+}
+
+/* Returns 0, or a negative code when the row's inputs are inconsistent. */
+static int decode_row(const oracle_problem *p, int64_t row, double *out, double *lse,
+                      double *scores) {
+    int h = (int)(row % p->H);
+    int t = (int)((row / p->H) % p->T);
+    int b = (int)(row / ((int64_t)p->H * p->T));
+    int ctx = p->ctx_lens[b];
+    int n = visible_count(p, b, t);
+    const uint16_t *ql = p->q_lat + row * ORACLE_DL;
+    const uint16_t *qp = p->q_pe + row * ORACLE_DR;
+
+    if (ctx < 0 || n < 0 || n > ctx) return -2;
+    for (int d = 0; d < ORACLE_DL; ++d) out[d] = 0.0;
+    if (n == 0) {
+        *lse = -INFINITY;
+        return 0;
+    }
+    /* scores s_j over the visible positions, through the page table */
+    for (int j = 0; j < n; ++j) {
+        int32_t page = p->page_table[(int64_t)b * p->page_table_stride + j / ORACLE_PAGE];
+        int slot = j % ORACLE_PAGE;
+        double dot = 0.0;
+        if (page < 0 || page >= p->num_pages) return -3;
+        for (int d = 0; d < ORACLE_DL; ++d)
+            dot += oracle_bf16_to_f64(ql[d]) * kv_value(p, page, slot, d);
+        for (int d = 0; d < ORACLE_DR; ++d)
+            dot += oracle_bf16_to_f64(qp[d]) * kv_value(p, page, slot, ORACLE_DL + d);
+        scores[j] = p->sm_scale * dot;
+    }
+    double M = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (scores[j] > M) M = scores[j];
+    double Z = 0.0;
+    for (int j = 0; j < n; ++j) Z += exp(scores[j] - M);
+    *lse = M + log(Z);
+    /* out = softmax-weighted sum of the latent part of the visible rows */
+    for (int j = 0; j < n; ++j) {
+        int32_t page = p->page_table[(int64_t)b * p->page_table_stride + j / ORACLE_PAGE];
+        int slot = j % ORACLE_PAGE;
+        double w = exp(scores[j] - M) / Z;
+        for (int d = 0; d < ORACLE_DL; ++d) out[d] += w * kv_value(p, page, slot, d);
+    }
+    return 0;
+}
+
+typedef struct {
+    const oracle_problem *p;
+    const int64_t *rows;     /* NULL: all rows */
+    int64_t n_rows;
+    double *out;
+    double *lse;
+    int64_t next;            /* shared work cursor */
+    pthread_mutex_t lock;
+    int status;
+    int max_ctx;
+} oracle_job;
+
+static void *worker(void *arg) {
+    oracle_job *job = (oracle_job *)arg;
+    double *scores = (double *)malloc(sizeof(double) * (size_t)(job->max_ctx > 0 ? job->max_ctx : 1));
+    for (;;) {
+        int64_t i;
+        pthread_mutex_lock(&job->lock);
+        i = job->next++;
+        pthread_mutex_unlock(&job->lock);
+        if (i >= job->n_rows) break;
+        int64_t row = job->rows ? job->rows[i] : i;
+        int rc = decode_row(job->p, row, job->out + i * ORACLE_DL, job->lse + i, scores);
+        if (rc) {
+            pthread_mutex_lock(&job->lock);
+            if (!job->status) job->status = rc;
+            pthread_mutex_unlock(&job->lock);
+        }
+    }
+    free(scores);
+    return NULL;
+}
+
+static int run_rows(const oracle_problem *p, const int64_t *rows, int64_t n_rows,
+                    double *out, double *lse, int n_threads) {
+    oracle_job job;
+    int max_ctx = 0;
+    int64_t total_rows = (int64_t)p->B * p->T * p->H;
+    if (p->B <= 0 || p->T <= 0 || p->H <= 0) return -1;
+    for (int b = 0; b < p->B; ++b)
+        if (p->ctx_lens[b] > max_ctx) max_ctx = p->ctx_lens[b];
+    for (int64_t i = 0; rows && i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= total_rows) return -1;
+    memset(&job, 0, sizeof job);
+    job.p = p;
+    job.rows = rows;
+    job.n_rows = n_rows;
+    job.out = out;
+    job.lse = lse;
+    job.max_ctx = max_ctx;
+    pthread_mutex_init(&job.lock, NULL);
+    if (n_threads <= 0) n_threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    pthread_t th[256];
+    for (int k = 0; k < n_threads; ++k) pthread_create(&th[k], NULL, worker, &job);
+    for (int k = 0; k < n_threads; ++k) pthread_join(th[k], NULL);
+    pthread_mutex_destroy(&job.lock);
+    return job.status;
+}
+
+/* Decode every row (rows == NULL) or the listed flat rows b*T*H + t*H + h.
+ * out: [n_rows, 512] fp64, lse: [n_rows] fp64.  Returns 0 on success. */
+int oracle_mla_decode(int B, int T, int H, const uint16_t *q_lat, const uint16_t *q_pe,
+                      const void *kv_pages, int kv_dtype, const float *kv_scale, int num_pages,
+                      const int32_t *page_table, int page_table_stride, const int32_t *ctx_lens,
+                      const int32_t *vis_lens, double sm_scale, const int64_t *rows,
+                      int64_t n_rows, double *out, double *lse, int n_threads) {
+    oracle_problem p;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.q_lat = q_lat;
+    p.q_pe = q_pe;
+    p.kv_pages = kv_pages;
+    p.kv_dtype = kv_dtype;
+    p.kv_scale = kv_scale;
+    p.num_pages = num_pages;
+    p.page_table = page_table;
+    p.page_table_stride = page_table_stride;
+    p.ctx_lens = ctx_lens;
+    p.vis_lens = vis_lens;
+    p.sm_scale = sm_scale;
+    if (kv_dtype != ORACLE_KV_BF16 && kv_dtype != ORACLE_KV_FP8) return -1;
+    if (kv_dtype == ORACLE_KV_FP8 && !kv_scale) return -1;
+    if (!rows) n_rows = (int64_t)B * T * H;
+    return run_rows(&p, rows, n_rows, out, lse, n_threads);
+}
+
+/* Merge n_parts partial results of the same rows, each normalised within its
+ * own part and carrying that part's log-sum-exp:
+ *   L = max_i lse_i,  w_i = exp(lse_i - L),  out = sum_i w_i out_i / sum_i w_i,
+ *   lse = L + ln sum_i w_i.
+ * Parts with lse = -inf weigh nothing; if every part is -inf the row is empty:
+ * out = 0, lse = -inf.  out_parts: [n_parts, rows, dv]; lse_parts: [n_parts, rows]. */
+int oracle_mla_merge(int n_parts, int64_t rows, int dv, const double *out_parts,
+                     const double *lse_parts, double *out, double *lse) {
+    if (n_parts <= 0 || rows < 0 || dv <= 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        double L = -INFINITY;
+        for (int i = 0; i < n_parts; ++i) {
+            double l = lse_parts[(int64_t)i * rows + r];
+            if (l > L) L = l;
+        }
+        double *o = out + r * dv;
+        for (int d = 0; d < dv; ++d) o[d] = 0.0;
+        if (L == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double W = 0.0;
+        for (int i = 0; i < n_parts; ++i) {
+            double l = lse_parts[(int64_t)i * rows + r];
+            if (l == -INFINITY) continue;
+            double w = exp(l - L);
+            const double *oi = out_parts + ((int64_t)i * rows + r) * dv;
+            W += w;
+            for (int d = 0; d < dv; ++d) o[d] += w * oi[d];
+        }
+        for (int d = 0; d < dv; ++d) o[d] /= W;
+        lse[r] = L + log(W);
+    }
+    return 0;
+}
