@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of paged MLA latent-attention decode on B200.
+
+One step = one decode step of a model's MLA stack: ``--layers`` (default 24)
+calls of ``mla_decode``, each over its own layer's paged KV cache, for the
+same batch of query rows.  24 layers x 142,000 positions x 576 FP8 bytes is
+the per-GPU MLA payload the Kimi K3 page quotes ("Inside Kimi K3 optimisation
+work", section 1, DCP), so the default workload, ``long_ctx_142k`` (B=1, T=1,
+H=96, 142,000 cached positions, FP8 e4m3 with per-token scale), reads 1.98 GB
+of KV per step; that is larger than the 126 MB L2, so every layer's cache
+comes from HBM.
+
+Prints one JSON line (rank 0).  ``value`` is KV-read GB/s of the whole job:
+the bytes of all cached positions each query row sees (read once per layer),
+over the device time of the timed steps.  ``--impl reference`` times the fp64
+CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import shutil
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mla_workloads as W  # noqa: E402
+
+METRIC = "MLA decode KV-read GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long_ctx_142k", choices=W.CONFIG_ORDER)
+    ap.add_argument("--kv", choices=[W.KV_BF16, W.KV_FP8], default=None)
+    ap.add_argument("--layers", type=int, default=24)
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# bookkeeping shared by both arms
+# ----------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def visible_positions(w) -> int:
+    """Sum over query rows' distinct sequences of cached positions read once
+    per layer (each sequence's pages are read once for all its rows)."""
+    return int(w.ctx_lens.to(torch.int64).sum())
+
+
+def step_units(w, layers):
+    pos = visible_positions(w)
+    kv_bytes = pos * w.kv_bytes_per_position() * layers
+    R = w.T * w.H
+    q_bytes = w.B * R * (512 + 64) * 2 * layers
+    out_bytes = w.B * R * (512 * 2 + 4) * layers
+    # flops: 2*576 (scores) + 2*512 (values) per (row, visible position)
+    if w.vis_lens is not None:
+        vis = int(w.vis_lens.to(torch.int64).sum()) * w.H
+    else:
+        ctx = w.ctx_lens.to(torch.int64)
+        vis = int(sum(int(c) - w.T + t + 1 for c in ctx for t in range(w.T))) * w.H
+    flops = 2176 * vis * layers
+    return dict(kv_bytes=kv_bytes, total_bytes=kv_bytes + q_bytes + out_bytes, flops=flops,
+                seqs=w.B)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        exe = shutil.which("nvidia-smi")
+        if exe is None:
+            return
+        self.proc = subprocess.Popen(
+            [exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+             "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[4:8]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * max(sm)]
+        busy.sort()
+        return {"sm_mhz": busy[len(busy) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, layers, seconds):
+    """Time the fp64 oracle on a bounded sample of rows of one layer.
+
+    Rows are taken whole (every visible position of each sampled row), in
+    batches of one row per core, until about ``seconds`` of wall time; the
+    time per full step is extrapolated by rows: layers * B*T*H / rows done."""
+    import oracle
+    lib = oracle.load()
+    wc = w.to("cpu")
+    total_rows = wc.B * wc.T * wc.H
+    threads = cpu_threads()
+    rows_done, t_spent, start = 0, 0.0, 0
+    gen = torch.Generator().manual_seed(5)
+    order = torch.randperm(total_rows, generator=gen)
+    while t_spent < seconds and rows_done < total_rows:
+        batch = order[start:start + threads]
+        start += threads
+        t0 = time.perf_counter()
+        oracle.decode_workload(wc, rows=batch, threads=threads, lib=lib)
+        t_spent += time.perf_counter() - t0
+        rows_done += int(batch.numel())
+    step_time = t_spent * layers * total_rows / rows_done
+    return step_time, rows_done, t_spent, threads
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the oracle on host cores
+# ----------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = W.make_workload(args.workload, kv=args.kv)
+    units = step_units(w, args.layers)
+    steps = args.steps if args.steps is not None else 3
+    budget = max(0.5, 120.0 / (steps + args.warmup))   # whole run within ~2 minutes
+    times = []
+    info = None
+    for i in range(args.warmup + steps):
+        st, rows, spent, threads = oracle_sample(w, args.layers, budget)
+        if i >= args.warmup:
+            times.append(st)
+            info = (rows, spent, threads)
+    step_time = sum(times) / len(times)
+    value = units["kv_bytes"] / step_time / 1e9
+    rows, spent, threads = info
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": step_time * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "T": w.T, "H": w.H, "kv": w.kv_dtype,
+                   "layers": args.layers},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} whole query rows of one layer per step "
+                                   f"({spent:.1f} s), extrapolated to {args.layers} layers x "
+                                   f"{w.B * w.T * w.H} rows"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import mla_latent_attention_b200 as mla
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.make_workload(args.workload, device=dev, kv=args.kv)
+    L = args.layers
+    units = step_units(w, L)
+    # each layer: its own copy of the paged cache (same contents, own memory)
+    kv = [w.kv_pages] + [w.kv_pages.clone() for _ in range(L - 1)]
+    sc = None if w.kv_scale is None else [w.kv_scale] + [w.kv_scale.clone() for _ in range(L - 1)]
+    B, T, H = w.B, w.T, w.H
+    q_lat = torch.stack([w.q_lat] * L)          # [L,B,T,H,512]
+    q_pe = torch.stack([w.q_pe] * L)
+    outs = torch.empty((L, B, T, H, 512), dtype=torch.bfloat16, device=dev)
+    lses = torch.empty((L, B, T, H), dtype=torch.float32, device=dev)
+    dims = mla.make_dims(w.q_lat, w.kv_pages, w.page_table, kernel=args.kernel,
+                         num_splits=args.num_splits)
+    ws_bytes = mla.workspace_size(dims)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    launches_per_call = 2 if ws_bytes > 256 else 1
+    ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
+    ev_m = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
+    ev_b = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
+
+    def one_step(timed_events):
+        for i in range(L):
+            if timed_events:
+                ev_a[i].record()
+            mla.decode(q_lat[i], q_pe[i], kv[i], None if sc is None else sc[i], w.page_table,
+                       w.ctx_lens, w.sm_scale, out=outs[i], lse=lses[i], kernel=args.kernel,
+                       num_splits=args.num_splits, workspace=ws,
+                       stage_event=ev_m[i] if timed_events else None)
+            if timed_events:
+                ev_b[i].record()
+
+    # eager warm-up (sets kernel attributes), then capture one step as a graph
+    one_step(False)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            one_step(True)
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    graph.replay()
+    torch.cuda.synchronize()
+    est = time.perf_counter() - t0
+    steps = args.steps if args.steps is not None else max(10, min(20000, int(3.0 / max(est, 1e-6))))
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    # keep the GPU busy ~0.5 s so clock samples reflect load, untimed
+    t_end = time.perf_counter() + 0.5
+    while time.perf_counter() < t_end:
+        graph.replay()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        graph.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed = start.elapsed_time(stop) / 1e3
+    # per-kernel durations of the last timed step (graph event nodes)
+    dec = [ev_a[i].elapsed_time(ev_m[i]) / 1e3 for i in range(L)]
+    mer = [ev_m[i].elapsed_time(ev_b[i]) / 1e3 for i in range(L)]
+    # plus a few more steps read one by one, for a steadier average
+    for _ in range(10):
+        graph.replay()
+        torch.cuda.synchronize()
+        dec += [ev_a[i].elapsed_time(ev_m[i]) / 1e3 for i in range(L)]
+        mer += [ev_m[i].elapsed_time(ev_b[i]) / 1e3 for i in range(L)]
+    clocks = sampler.stop()
+
+    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_elapsed = float(t.item())
+
+    # end to end through the public API with host buffers: per step the query
+    # rows of every layer go host->device and the outputs come back.
+    h_qlat = torch.empty(q_lat.shape, dtype=q_lat.dtype, pin_memory=True).copy_(q_lat)
+    h_qpe = torch.empty(q_pe.shape, dtype=q_pe.dtype, pin_memory=True).copy_(q_pe)
+    h_out = torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True)
+    h_lse = torch.empty(lses.shape, dtype=lses.dtype, pin_memory=True)
+    e2e_steps = max(3, min(steps, 200))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        q_lat.copy_(h_qlat, non_blocking=True)
+        q_pe.copy_(h_qpe, non_blocking=True)
+        one_step(False)
+        h_out.copy_(outs, non_blocking=True)
+        h_lse.copy_(lses, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_t = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = world * e2e_steps * units["kv_bytes"] / float(e2e_t.item()) / 1e9
+    h2d = (h_qlat.numel() * h_qlat.element_size() + h_qpe.numel() * h_qpe.element_size())
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    value = world * steps * units["kv_bytes"] / max_elapsed / 1e9
+    dec_avg = sum(dec) / len(dec)
+    per_launch_bytes = units["total_bytes"] / L
+    per_launch_flops = units["flops"] / L
+    achieved_gbs = per_launch_bytes / dec_avg / 1e9
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": None,
+                "kernel": "mla decode attention kernel", "peak_source": f"{peak_src} hbm_gbs",
+                "avg_launch_us": dec_avg * 1e6, "merge_avg_launch_us": sum(mer) / len(mer) * 1e6}
+    tflops = per_launch_flops / dec_avg / 1e12
+    kernel_dtype = {"simt": "f32"}.get(args.kernel, "e4m3" if w.kv_dtype == W.KV_FP8 else "bf16")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": max_elapsed / steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": kernel_dtype, "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "T": T, "H": H,
+                   "ctx": int(w.ctx_lens.max()), "kv": w.kv_dtype, "layers": L,
+                   "kernel": args.kernel, "num_splits": args.num_splits,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {L} layer caches, "
+                         f"{units['kv_bytes'] / 1e9:.2f} GB of KV per step"},
+        "hbm_fraction_of_8TBs": value / world / NOMINAL_HBM_GBS,
+        "seq_steps_per_s": world * steps * units["seqs"] / max_elapsed,
+        "tensor_tflops": tflops,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": steps * L * launches_per_call,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        st, rows, spent, threads = oracle_sample(w, L, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": units["kv_bytes"] / st / 1e9, "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{rows} whole query rows of one layer ({spent:.1f} s), extrapolated to "
+                      f"{L} layers x {B * T * H} rows"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        if args.impl == "ours":
+            torch.cuda.set_device(local_rank)
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

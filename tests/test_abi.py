@@ -1,0 +1,113 @@
+"""The C-ABI library builds, loads and exports its declared symbols; host-side
+argument checks return the documented status codes without touching a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import mla_latent_attention_b200 as mla
+from mla_latent_attention_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names.update(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return mla.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    assert {"mla_decode", "mla_merge_partials", "mla_decode_workspace_size"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", mla.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)", out))
+    missing = _declared() - exported
+    assert not missing, f"declared but not exported: {missing}"
+    for name in _declared():
+        assert hasattr(lib, name)
+    assert set(mla.EXPORTED) <= exported
+
+
+def test_library_is_sm100a_only():
+    """The fatbinary is built for sm_100a (checked on the build command, not the binary)."""
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def _dims(**kw):
+    d = dict(B=1, T=1, H=16, num_pages=16, max_pages_per_seq=16, page_table_stride=16,
+             kv_dtype=0, out_dtype=0, num_splits=0, kernel=0, vis_lens=None, stage_event=None)
+    d.update(kw)
+    return mla.Dims(**d)
+
+
+BAD_DIMS = [dict(B=0), dict(T=0), dict(T=9), dict(H=0), dict(T=8, H=129), dict(num_pages=0),
+            dict(max_pages_per_seq=0), dict(page_table_stride=8), dict(kv_dtype=2),
+            dict(out_dtype=5), dict(num_splits=-1), dict(kernel=7)]
+
+
+@pytest.mark.parametrize("bad", BAD_DIMS, ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))
+def test_invalid_dims_rejected_without_gpu(lib, bad):
+    d = _dims(**bad)
+    assert lib.mla_decode_workspace_size(ctypes.byref(d)) == -1
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) & ~255)
+    rc = lib.mla_decode(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), p, 4096, None)
+    assert rc == -1
+
+
+def test_null_pointers_rejected_without_gpu(lib):
+    d = _dims()
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) & ~255)
+    assert lib.mla_decode(None, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), p, 4096, None) == -1
+    assert lib.mla_decode(p, p, p, None, p, None, 0.1, p, None, ctypes.byref(d), p, 4096, None) == -1
+    # FP8 needs kv_scale, bf16 must not have one
+    d8 = _dims(kv_dtype=1)
+    assert lib.mla_decode(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(d8), p, 4096, None) == -1
+    assert lib.mla_decode(p, p, p, p, p, p, 0.1, p, None, ctypes.byref(d), p, 4096, None) == -1
+    # misaligned KV pool
+    q = ctypes.c_void_p(p.value + 8)
+    assert lib.mla_decode(p, p, q, None, p, p, 0.1, p, None, ctypes.byref(d), p, 4096, None) == -1
+    # non-finite softmax scale
+    assert lib.mla_decode(p, p, p, None, p, p, float("nan"), p, None, ctypes.byref(d), p, 4096, None) == -1
+    # workspace missing or misaligned
+    assert lib.mla_decode(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), None, 4096, None) == -3
+    assert lib.mla_decode(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), q, 4096, None) == -3
+
+
+def test_merge_argument_checks_without_gpu(lib):
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) & ~255)
+    assert lib.mla_merge_partials(None, p, 2, 4, p, 0, None, None) == -1
+    assert lib.mla_merge_partials(p, p, 0, 4, p, 0, None, None) == -1
+    assert lib.mla_merge_partials(p, p, 4097, 4, p, 0, None, None) == -1
+    assert lib.mla_merge_partials(p, p, 2, -1, p, 0, None, None) == -1
+    assert lib.mla_merge_partials(p, p, 2, 4, p, 3, None, None) == -1
+    assert lib.mla_merge_partials(ctypes.c_void_p(p.value + 4), p, 2, 4, p, 0, None, None) == -1
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4):
+        assert lib.mla_status_string(code)
+    assert lib.mla_status_string(-99) == b"unknown status"
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(mla.MlaError):
+        mla.load_library(str(tmp_path / "missing.so"))
