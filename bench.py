@@ -92,6 +92,27 @@ def step_units(w, layers):
                 seqs=w.B)
 
 
+_LIBCUDA = None
+
+
+def event_ms(a, b) -> float:
+    """Elapsed ms between two recorded CUDA events, through the driver API
+    (works for event-record nodes of a replayed CUDA graph, which torch's
+    Event.elapsed_time refuses)."""
+    import ctypes
+    global _LIBCUDA
+    if _LIBCUDA is None:
+        _LIBCUDA = ctypes.CDLL("libcuda.so.1")
+        _LIBCUDA.cuEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p,
+                                                ctypes.c_void_p]
+    ms = ctypes.c_float(0.0)
+    rc = _LIBCUDA.cuEventElapsedTime(ctypes.byref(ms), ctypes.c_void_p(a.cuda_event),
+                                     ctypes.c_void_p(b.cuda_event))
+    if rc != 0:
+        raise RuntimeError(f"cuEventElapsedTime failed with CUresult {rc}")
+    return float(ms.value)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -253,6 +274,10 @@ def run_ours(args, rank, world, local_rank):
             if timed_events:
                 ev_b[i].record()
 
+    # torch creates CUDA events lazily: record each once so its handle exists
+    # before it is handed to the library or captured
+    for e in ev_a + ev_m + ev_b:
+        e.record()
     # eager warm-up (sets kernel attributes), then capture one step as a graph
     one_step(False)
     torch.cuda.synchronize()
@@ -290,14 +315,14 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     elapsed = start.elapsed_time(stop) / 1e3
     # per-kernel durations of the last timed step (graph event nodes)
-    dec = [ev_a[i].elapsed_time(ev_m[i]) / 1e3 for i in range(L)]
-    mer = [ev_m[i].elapsed_time(ev_b[i]) / 1e3 for i in range(L)]
+    dec = [event_ms(ev_a[i], ev_m[i]) / 1e3 for i in range(L)]
+    mer = [event_ms(ev_m[i], ev_b[i]) / 1e3 for i in range(L)]
     # plus a few more steps read one by one, for a steadier average
     for _ in range(10):
         graph.replay()
         torch.cuda.synchronize()
-        dec += [ev_a[i].elapsed_time(ev_m[i]) / 1e3 for i in range(L)]
-        mer += [ev_m[i].elapsed_time(ev_b[i]) / 1e3 for i in range(L)]
+        dec += [event_ms(ev_a[i], ev_m[i]) / 1e3 for i in range(L)]
+        mer += [event_ms(ev_m[i], ev_b[i]) / 1e3 for i in range(L)]
     clocks = sampler.stop()
 
     t = torch.tensor([elapsed], dtype=torch.float64, device=dev)

@@ -87,7 +87,8 @@ typedef enum {
     MLA_DEV_OK = 0,
     MLA_DEV_BAD_PAGE = 1,   /* page_table entry outside [0, num_pages); info = sequence */
     MLA_DEV_BAD_CTX = 2,    /* ctx_lens[b] < 0, > max_pages_per_seq*16, or < T without vis_lens; info = b */
-    MLA_DEV_BAD_VIS = 3     /* vis_lens[b,t] < 0 or > ctx_lens[b]; info = b*T + t */
+    MLA_DEV_BAD_VIS = 3,    /* vis_lens[b,t] < 0 or > ctx_lens[b]; info = b*T + t */
+    MLA_DEV_TIMEOUT = 4     /* a bounded on-chip wait gave up (the CTA stopped cleanly); info = CTA */
 } mla_device_error;
 
 typedef struct mla_dims {
@@ -125,7 +126,8 @@ MLA_API int64_t mla_decode_workspace_size(const mla_dims *dims);
  *                                   are c_kv (also the attention value),
  *                                   512..575 are k_pe.  16-byte aligned.
  *   kv_scale   [P,16] fp32          FP8 only: dequantised value = e4m3 * scale
- *                                   of its position.  Must be NULL for bf16.
+ *                                   of its position.  16-byte aligned.  Must be
+ *                                   NULL for bf16.
  *   page_table [B, stride] int32    page_table[b][i] = physical page of the
  *                                   sequence's positions 16i .. 16i+15.  Only
  *                                   entries i < ceil(ctx_lens[b]/16) are read.

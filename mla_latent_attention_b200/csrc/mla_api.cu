@@ -60,7 +60,7 @@ int make_plan(const mla_dims *d, Plan *pl) {
     int sms = 0;
     rc = device_sm_count(&sms);
     if (rc) return rc;
-    pl->kernel = d->kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_SIMT : d->kernel;
+    pl->kernel = d->kernel == MLA_KERNEL_AUTO ? MLA_KERNEL_TCGEN05 : d->kernel;
     pl->rows_per_group = pl->kernel == MLA_KERNEL_SIMT ? kSimtRows : kTcRows;
     const int R = d->T * d->H;
     pl->n_groups = (R + pl->rows_per_group - 1) / pl->rows_per_group;
@@ -109,7 +109,7 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     if (!q_lat || !q_pe || !kv_pages || !page_table || !ctx_lens || !out) return MLA_ERR_INVALID_ARG;
     if ((dims->kv_dtype == MLA_KV_FP8_E4M3) != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
     if (!aligned(q_lat, 16) || !aligned(q_pe, 16) || !aligned(kv_pages, 16) || !aligned(out, 16) ||
-        !aligned(page_table, 4) || !aligned(ctx_lens, 4) || (kv_scale && !aligned(kv_scale, 4)) ||
+        !aligned(page_table, 4) || !aligned(ctx_lens, 4) || (kv_scale && !aligned(kv_scale, 16)) ||
         (lse && !aligned(lse, 4)))
         return MLA_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || sm_scale == INFINITY || sm_scale == -INFINITY) return MLA_ERR_INVALID_ARG;

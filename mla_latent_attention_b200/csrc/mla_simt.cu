@@ -98,9 +98,13 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(Problem p) {
                 piece_ok = false;
                 if (tid == 0) report_error(p.err, MLA_DEV_BAD_PAGE, pc.b);
             } else {
+                // Slots past the context hold undefined data (possibly NaN);
+                // they get zero weight, and 0 * NaN would still poison the
+                // value sum, so they are staged as zeros.
+                const int valid = pc.ctx - pg * kPage;
                 for (int i = tid; i < kPage * kD; i += kThreads) {
                     int s = i / kD, d = i % kD;
-                    sm.kv[s][d] = load_kv(p, kFp8, (int64_t)page * kPage + s, d);
+                    sm.kv[s][d] = s < valid ? load_kv(p, kFp8, (int64_t)page * kPage + s, d) : 0.f;
                 }
             }
             __syncthreads();

@@ -1,6 +1,812 @@
-// tcgen05 tensor-core decode kernel (not built yet).
+// tcgen05 tensor-core decode kernel for B200 (sm_100a).
+//
+// One CTA = one (KV range, group of 48 query rows).  Query rows are the
+// heads x draft tokens of one sequence, packed together (12 heads x 3 tokens
+// = 36 rows fill one group; 96 x 3 = 288 rows make six), so the padding of
+// odd head counts exists only on chip.  The CTA walks its range in tiles of
+// 128 cached positions (8 pages of 16).
+//
+// Orientation ("swap AB"): positions are the MMA M dimension (128 TMEM lanes)
+// and query rows the N dimension (48 columns), so
+//     S^T [128 x 48] = KV_tile[128 x 576] . Q^T          (scores)
+//     O^T [512 x 48] += V_tile^T[512 x 128] . P^T         (values, 4 blocks of 128)
+// S^T (two buffers) and O^T live in tensor memory: 2*48 + 4*48 columns of
+// the 512.  With the rows as M instead, a 128 x 512 fp32 O alone would fill
+// all of tensor memory.
+//
+// FP8 caches are consumed as stored, by kind::f8f6f4 MMAs:
+//   * scores: the query is split on chip into two e4m3 parts, hi = e4m3(q/s)
+//     and lo = e4m3(q/s - hi), with one power-of-two scale s per CTA, and S
+//     accumulates K.hi + K.lo.  For a bf16 query hi + lo is exact (a bf16
+//     significand has 8 bits, hi takes the top 4 and the remainder fits lo),
+//     at the tensor-core cost of one bf16 MMA; the per-token scale multiplies
+//     S^T lane by lane.
+//   * values: P^T is split the same way into two e4m3 operands, after the
+//     per-token value scale has been folded into each weight, so V is read
+//     as stored and never dequantised.
+// bf16 caches use kind::f16 MMAs with bf16 P.
+//
+// Warp roles (192 threads): warp 0 issues TMA page loads, warp 1 issues the
+// MMAs and owns tensor memory, warps 2-5 (one per TMEM lane quadrant) run the
+// online softmax and the epilogue; thread (warp w, lane l) owns tile position
+// / TMEM lane 32*(w%4) + l.
+//
+// Softmax stabiliser: per query row a running bound m2 on the log2 weight
+// u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
+// all lanes.  It moves only when some weight exceeds it by more than TAU
+// (then O^T and the row sums are rescaled), which after the first tile is
+// rare.  Weights are exp2(u - m2 + C), at most 2^(TAU+C), chosen to stay in
+// the e4m3 range for FP8.  Row sums are kept per lane and reduced once per
+// piece.
+//
+// Every wait is bounded: after two seconds the CTA records a timeout in the
+// error word, stops, drains its outstanding copies and MMAs and frees its
+// tensor memory.
+#include <cuda.h>
+#include <cuda_fp8.h>
+#include <cudaTypedefs.h>
+
 #include "mla_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace mla {
-int launch_tc(const Problem &, cudaStream_t) { return MLA_ERR_UNSUPPORTED; }
+namespace {
+
+constexpr int kN = 48;            // query rows per CTA (MMA N)
+constexpr int kTileM = 128;       // positions per tile (MMA M)
+constexpr int kTilePages = kTileM / kPage;
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;  // O block m at kColO + 64m
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kDevTimeout = 4;
+
+template <bool kFp8>
+struct Cfg {
+    static constexpr int kStages = kFp8 ? 2 : 1;
+    // KV stage: chunks of [128 positions][128 B], plus for FP8 the RoPE chunk [128][64 B]
+    static constexpr int kChunkBytes = kTileM * 128;                              // 16384
+    static constexpr int kVChunks = kFp8 ? 4 : 8;                                 // chunks holding c_kv
+    static constexpr int kStageBytes = kFp8 ? 4 * kChunkBytes + kTileM * 64 : 9 * kChunkBytes;
+    static constexpr int kKvOff = 0;
+    static constexpr int kScaleOff = kKvOff + kStages * kStageBytes;               // FP8: 512 B / stage
+    static constexpr int kScaleBytes = kFp8 ? kTileM * 4 : 0;
+    static constexpr int kQOff = (kScaleOff + kStages * kScaleBytes + 1023) & ~1023;
+    static constexpr int kQChunk = kN * 128;                                       // 6144
+    static constexpr int kQPart = kFp8 ? 4 * kQChunk + kN * 64 : 9 * kQChunk;      // one operand
+    static constexpr int kQBytes = kFp8 ? 2 * kQPart : kQPart;
+    static constexpr int kPOff = (kQOff + kQBytes + 1023) & ~1023;
+    static constexpr int kPGroupRows = kFp8 ? 16 : 8;                              // rows per 16 B
+    static constexpr int kPPart = (kN / kPGroupRows) * kTileM * 16;                // one P operand
+    static constexpr int kPBytes = kFp8 ? 2 * kPPart : kPPart;                     // FP8: hi and lo
+    static constexpr int kMiscOff = kPOff + kPBytes;
+    static constexpr int kPageBytes = kFp8 ? (4 * 2048 + 1024 + 64) : 9 * 2048;   // bytes a page brings
+    // exponent offset C and lazy threshold TAU of the softmax stabiliser
+    static constexpr float kC = kFp8 ? 6.5f : 0.f;
+    static constexpr float kTau = kFp8 ? 2.f : 8.f;
+};
+
+struct Misc {
+    uint64_t kv_full[2], kv_empty[2], s_full[2], s_free[2];
+    uint64_t p_full, pv_done, q_ready, o_free, drain;
+    uint64_t group;           // barrier of the four softmax warps (bounded, unlike bar.sync)
+    uint32_t tmem_base;
+    int abort;
+    uint32_t stage_info[2];   // bit i: page slot i loaded; bit 31: a page of the tile was invalid
+    int vote[2][4];
+    int col_lim[kN];          // positions visible to column r within this piece, 0 = none
+    int col_bad[kN];
+    float qscale;
+    float red[4][kN];
+    float m2[kN];
+    float inv_l[kN];
+    float lse[kN];
+};
+
+template <bool kFp8>
+constexpr int smem_bytes() {
+    return Cfg<kFp8>::kMiscOff + (int)sizeof(Misc) + 1024;  // + alignment slack
+}
+
+__device__ __forceinline__ void cta_abort(const Problem &p, Misc &ms) {
+    if (atomicExch(&ms.abort, 1) == 0) report_error(p.err, kDevTimeout, blockIdx.x);
+}
+
+__device__ __forceinline__ bool aborted(Misc &ms) { return *reinterpret_cast<volatile int *>(&ms.abort) != 0; }
+
+__device__ __forceinline__ bool waitb(const Problem &p, Misc &ms, uint64_t *bar, uint32_t parity) {
+    if (ptx::mbar_wait(bar, parity, kWaitLimitNs)) return true;
+    cta_abort(p, ms);
+    return false;
+}
+
+// Barrier of the four softmax warps.  An mbarrier with a bounded wait: if a
+// warp has stopped on a timeout, the others give up too instead of hanging.
+struct GroupSync {
+    uint32_t phase = 0;
+    __device__ __forceinline__ bool operator()(const Problem &p, Misc &ms) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&ms.group);
+        const bool ok = waitb(p, ms, &ms.group, phase & 1);
+        ++phase;
+        return ok;
+    }
+};
+
+__device__ __forceinline__ int ntiles_of(const Piece &pc) {
+    return (pc.page_hi - pc.page_lo + kTilePages - 1) / kTilePages;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Query split for the e4m3 score MMA: hi = e4m3(x), lo = e4m3(x - hi), so that
+// hi + lo carries about twice the mantissa bits of one e4m3 value.
+__device__ __forceinline__ void split_e4m3(float x, uint8_t &hi, uint8_t &lo) {
+    const __nv_fp8_e4m3 h(x);              // round to nearest, saturating
+    const __nv_fp8_e4m3 l(x - float(h));
+    hi = h.__x;
+    lo = l.__x;
+}
+
+// ---------------------------------------------------------------------------
+// warp 0: TMA producer
+// ---------------------------------------------------------------------------
+template <bool kFp8>
+__device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUtensorMap *map_b,
+                         unsigned char *smem, Misc &ms, int slot) {
+    using C = Cfg<kFp8>;
+    const int lane = threadIdx.x & 31;
+    uint32_t g = 0;
+    for_each_piece(p, slot, [&](const Piece &pc) {
+        const int nt = ntiles_of(pc);
+        for (int k = 0; k < nt; ++k, ++g) {
+            if (aborted(ms)) return;
+            const int stage = g % C::kStages;
+            if (!waitb(p, ms, &ms.kv_empty[stage], ((g / C::kStages) & 1) ^ 1)) return;
+            const int pg0 = pc.page_lo + k * kTilePages;
+            const int npg = min(kTilePages, pc.page_hi - pg0);
+            int pid = -1;
+            bool ok = false;
+            if (lane < npg) {
+                pid = __ldg(p.page_table + (int64_t)pc.b * p.pt_stride + pg0 + lane);
+                ok = pid >= 0 && pid < p.num_pages;
+            }
+            const unsigned okm = __ballot_sync(0xffffffffu, ok);
+            const unsigned badm = __ballot_sync(0xffffffffu, lane < npg && !ok);
+            if (lane == 0) {
+                if (badm) report_error(p.err, MLA_DEV_BAD_PAGE, pc.b);
+                ms.stage_info[stage] = okm | (badm ? 0x80000000u : 0u);
+                ptx::mbar_arrive_expect_tx(&ms.kv_full[stage], __popc(okm) * C::kPageBytes);
+            }
+            __syncwarp();
+            if (ok) {
+                unsigned char *st = smem + C::kKvOff + stage * C::kStageBytes;
+                const int y = pid * kPage;
+                if constexpr (kFp8) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        ptx::tma_load_2d(st + c * C::kChunkBytes + lane * 2048, map_a, &ms.kv_full[stage],
+                                         128 * c, y);
+                    ptx::tma_load_2d(st + 4 * C::kChunkBytes + lane * 1024, map_b, &ms.kv_full[stage], 512, y);
+                    ptx::bulk_load(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
+                                   p.kv_scale + (int64_t)pid * kPage, 64, &ms.kv_full[stage]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 9; ++c)
+                        ptx::tma_load_2d(st + c * C::kChunkBytes + lane * 2048, map_a, &ms.kv_full[stage],
+                                         64 * c, y);
+                }
+            }
+        }
+    });
+    // make sure no copy is still landing when the CTA leaves
+    for (uint32_t h = g > (uint32_t)C::kStages ? g - C::kStages : 0; h < g; ++h)
+        ptx::mbar_wait(&ms.kv_full[h % C::kStages], (h / C::kStages) & 1, kWaitLimitNs);
+}
+
+// ---------------------------------------------------------------------------
+// warp 1: MMA issuer
+// ---------------------------------------------------------------------------
+template <bool kFp8>
+__device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int slot) {
+    using C = Cfg<kFp8>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t tmem = ms.tmem_base;
+    const uint32_t kv0 = ptx::smem_u32(smem + C::kKvOff);
+    const uint32_t q0 = ptx::smem_u32(smem + C::kQOff);
+    const uint32_t p0 = ptx::smem_u32(smem + C::kPOff);
+    constexpr uint32_t idesc_qk = kFp8 ? ptx::instr_desc(0, 0, 0, 0, kTileM, kN)
+                                       : ptx::instr_desc(1, 1, 0, 0, kTileM, kN);
+    constexpr uint32_t idesc_pv = kFp8 ? ptx::instr_desc(0, 0, 1, 1, kTileM, kN)
+                                       : ptx::instr_desc(1, 1, 1, 1, kTileM, kN);
+    uint32_t g = 0, pi = 0;
+
+    auto issue_qk = [&](uint32_t gg) {
+        const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
+        const uint32_t d = tmem + ((gg & 1) ? kColS1 : kColS0);
+        if constexpr (kFp8) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t qb = q0 + part * C::kQPart;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        uint64_t a = ptx::smem_desc(st + c * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                        uint64_t b = ptx::smem_desc(qb + c * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                        ptx::mma_f8(d, a, b, idesc_qk, acc);
+                        acc = 1;
+                    }
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint64_t a = ptx::smem_desc(st + 4 * C::kChunkBytes + ks * 32, 16, 512, ptx::kSwizzle64B);
+                    uint64_t b = ptx::smem_desc(qb + 4 * C::kQChunk + ks * 32, 16, 512, ptx::kSwizzle64B);
+                    ptx::mma_f8(d, a, b, idesc_qk, 1);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 9; ++c)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint64_t a = ptx::smem_desc(st + c * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    uint64_t b = ptx::smem_desc(q0 + c * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    ptx::mma_f16(d, a, b, idesc_qk, (c | ks) ? 1u : 0u);
+                }
+        }
+    };
+
+    auto issue_pv = [&](uint32_t gg, bool first) {
+        const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t d = tmem + kColO + 64 * m;
+            if constexpr (kFp8) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {  // 32 positions per MMA; P = hi + lo
+                    uint64_t a = ptx::smem_desc(st + m * C::kChunkBytes + ks * 4096, 16384, 1024, ptx::kSwizzle128B);
+                    uint64_t bh = ptx::smem_desc(p0 + ks * 512, 128, 2048, ptx::kSwizzleNone);
+                    uint64_t bl = ptx::smem_desc(p0 + C::kPPart + ks * 512, 128, 2048, ptx::kSwizzleNone);
+                    ptx::mma_f8(d, a, bh, idesc_pv, (first && ks == 0) ? 0u : 1u);
+                    ptx::mma_f8(d, a, bl, idesc_pv, 1u);
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {  // 16 positions per MMA
+                    uint64_t a = ptx::smem_desc(st + 2 * m * C::kChunkBytes + ks * 2048, 16384, 1024,
+                                                ptx::kSwizzle128B);
+                    uint64_t b = ptx::smem_desc(p0 + ks * 256, 128, 2048, ptx::kSwizzleNone);
+                    ptx::mma_f16(d, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
+                }
+            }
+        }
+    };
+
+    for_each_piece(p, slot, [&](const Piece &pc) {
+        const int nt = ntiles_of(pc);
+        if (nt == 0 || aborted(ms)) return;
+        if (!waitb(p, ms, &ms.q_ready, pi & 1)) return;
+        ptx::tc_fence_after();
+        const uint32_t g0 = g;
+        auto do_qk = [&](int k) -> bool {
+            const uint32_t gg = g0 + k;
+            if (!waitb(p, ms, &ms.kv_full[gg % C::kStages], (gg / C::kStages) & 1)) return false;
+            if (!waitb(p, ms, &ms.s_free[gg & 1], ((gg >> 1) & 1) ^ 1)) return false;
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                issue_qk(gg);
+                ptx::mma_commit(&ms.s_full[gg & 1]);
+            }
+            __syncwarp();
+            return true;
+        };
+        auto do_pv = [&](int k) -> bool {
+            const uint32_t gp = g0 + k;
+            if (!waitb(p, ms, &ms.p_full, gp & 1)) return false;
+            if (k == 0 && !waitb(p, ms, &ms.o_free, (pi & 1) ^ 1)) return false;
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                issue_pv(gp, k == 0);
+                ptx::mma_commit(&ms.kv_empty[gp % C::kStages]);
+                ptx::mma_commit(&ms.pv_done);
+            }
+            __syncwarp();
+            return true;
+        };
+        // With two KV stages the scores of tile k are issued before the values
+        // of tile k-1, so the tensor core works while the softmax runs; with
+        // one stage, tile k can only land after tile k-1's values are done.
+        for (int k = 0; k <= nt; ++k) {
+            if (C::kStages > 1) {
+                if (k < nt && !do_qk(k)) return;
+                if (k > 0 && !do_pv(k - 1)) return;
+            } else {
+                if (k > 0 && !do_pv(k - 1)) return;
+                if (k < nt && !do_qk(k)) return;
+            }
+        }
+        g = g0 + nt;
+        ++pi;
+    });
+    // every MMA issued has completed before tensor memory is released
+    if (lane == 0) ptx::mma_commit(&ms.drain);
+    __syncwarp();
+    ptx::mbar_wait(&ms.drain, 0, kWaitLimitNs);
+}
+
+// ---------------------------------------------------------------------------
+// warps 2-5: query staging, online softmax, epilogue
+// ---------------------------------------------------------------------------
+template <bool kFp8>
+__device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int b, int r0, int st,
+                           GroupSync &gsync) {
+    using C = Cfg<kFp8>;
+    const int64_t qrow0 = (int64_t)b * p.R;
+    unsigned char *qs = smem + C::kQOff;
+    if constexpr (kFp8) {
+        // pass 1: the block's largest |q| sets the e4m3 scale
+        float amax = 0.f;
+        for (int u = st; u < kN * 36; u += kSoftmaxThreads) {
+            const int row = u / 36, uu = u % 36;
+            if (r0 + row >= p.R) continue;
+            const __nv_bfloat16 *src = uu < 32 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 16
+                                               : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 32) * 16;
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint4 v = __ldg(s4 + h);
+                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 f = __bfloat1622float2(b2[e]);
+                    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                }
+            }
+        }
+        amax = warp_max(amax);
+        const int w = (threadIdx.x >> 5) - 2;
+        if ((threadIdx.x & 31) == 0) ms.red[w][0] = amax;
+        if (!gsync(p, ms)) return false;
+        amax = fmaxf(fmaxf(ms.red[0][0], ms.red[1][0]), fmaxf(ms.red[2][0], ms.red[3][0]));
+        // A power-of-two scale keeps q/s a bf16 value, which hi + lo then
+        // represents exactly (short of e4m3 underflow far below the largest q).
+        int e2 = 0;
+        if (amax > 0.f) frexpf(amax / 448.f, &e2);
+        const float qscale = ldexpf(1.f, e2);
+        const float inv = ldexpf(1.f, -e2);
+        if (st == 0) ms.qscale = qscale;
+        // pass 2: hi = e4m3(q/s), lo = e4m3(q/s - hi), in the MMA's K-major layouts
+        for (int u = st; u < kN * 36; u += kSoftmaxThreads) {
+            const int row = u / 36, uu = u % 36;
+            uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
+            if (r0 + row < p.R) {
+                const __nv_bfloat16 *src = uu < 32 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 16
+                                                   : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 32) * 16;
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+                uint8_t *hv = reinterpret_cast<uint8_t *>(&hi4);
+                uint8_t *lv = reinterpret_cast<uint8_t *>(&lo4);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint4 v = __ldg(s4 + h);
+                    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(b2[e]);
+                        split_e4m3(f.x * inv, hv[8 * h + 2 * e], lv[8 * h + 2 * e]);
+                        split_e4m3(f.y * inv, hv[8 * h + 2 * e + 1], lv[8 * h + 2 * e + 1]);
+                    }
+                }
+            }
+            int off;
+            if (uu < 32) {
+                const int c = uu >> 3, k = uu & 7;
+                off = c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4);
+            } else {
+                const int k = uu - 32;
+                off = 4 * C::kQChunk + row * 64 + ((k ^ ((row >> 1) & 3)) << 4);
+            }
+            *reinterpret_cast<uint4 *>(qs + off) = hi4;
+            *reinterpret_cast<uint4 *>(qs + C::kQPart + off) = lo4;
+        }
+    } else {
+        for (int u = st; u < kN * 72; u += kSoftmaxThreads) {
+            const int row = u / 72, uu = u % 72;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r0 + row < p.R) {
+                const __nv_bfloat16 *src = uu < 64 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 8
+                                                   : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 64) * 8;
+                v = __ldg(reinterpret_cast<const uint4 *>(src));
+            }
+            const int c = uu >> 3, k = uu & 7;
+            *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4)) = v;
+        }
+    }
+    return true;
+}
+
+template <bool kFp8>
+__device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, int slot, int g_idx) {
+    using C = Cfg<kFp8>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int i = quad * 32 + lane;            // tile position / TMEM lane
+    const int st = threadIdx.x - 64;           // 0..127 for cooperative loops
+    const int wi = warp - 2;                   // 0..3 slot in reduction buffers
+    const uint32_t tmem = ms.tmem_base + ((uint32_t)(quad * 32) << 16);
+    const int r0 = g_idx * kN;
+    uint32_t g = 0, pi = 0;
+    GroupSync gsync;
+
+    for_each_piece(p, slot, [&](const Piece &pc) {
+        if (aborted(ms)) return;
+        const int nt = ntiles_of(pc);
+        // visible positions per column, limited to this piece's pages
+        if (st < kN) {
+            const int r = r0 + st;
+            int lim = 0, bad = 0;
+            if (pc.bad_ctx) {
+                bad = 1;
+            } else if (r < p.R) {
+                const int v = visible(p, pc.b, r / p.H, pc.ctx);
+                if (v < 0) {
+                    bad = 1;
+                    if (r % p.H == 0 || st == 0) report_error(p.err, MLA_DEV_BAD_VIS, pc.b * p.T + r / p.H);
+                } else {
+                    lim = min(v, pc.page_hi * kPage);
+                }
+            }
+            ms.col_lim[st] = lim;
+            ms.col_bad[st] = bad;
+        }
+        if (st == 0 && pc.bad_ctx && g_idx == 0) report_error(p.err, MLA_DEV_BAD_CTX, pc.b);
+        if (!gsync(p, ms)) return;
+        const int rows_here = min(kN, p.R - r0);
+        int min_lim = INT_MAX;
+        for (int c = 0; c < rows_here; ++c) min_lim = min(min_lim, ms.col_lim[c]);
+
+        if (nt == 0) {  // nothing to read: write the empty (or invalid) result
+            for (int e = st; e < rows_here * kDl; e += kSoftmaxThreads) {
+                const int c = e / kDl, d = e % kDl;
+                const bool bad = ms.col_bad[c] != 0;
+                store_out(p.out, ((int64_t)pc.b * p.R + r0 + c) * kDl + d, bad ? NAN : 0.f, p.out_f32);
+                if (d == 0 && p.lse) p.lse[(int64_t)pc.b * p.R + r0 + c] = bad ? NAN : -INFINITY;
+            }
+            gsync(p, ms);
+            return;
+        }
+
+        if (!load_query<kFp8>(p, smem, ms, pc.b, r0, st, gsync)) return;
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&ms.q_ready);
+        if (!gsync(p, ms)) return;  // qscale visible
+        const float qscale = kFp8 ? ms.qscale : 1.f;
+
+        float m2[kN], lsum[kN];
+#pragma unroll
+        for (int c = 0; c < kN; ++c) {
+            m2[c] = -INFINITY;
+            lsum[c] = 0.f;
+        }
+        bool piece_bad = false;
+        const uint32_t g0 = g;
+        for (int k = 0; k < nt; ++k) {
+            const uint32_t gg = g0 + k;
+            const int stage = gg % C::kStages;
+            if (!waitb(p, ms, &ms.kv_full[stage], (gg / C::kStages) & 1)) return;
+            const uint32_t info = ms.stage_info[stage];
+            piece_bad |= (info >> 31) != 0;
+            if (!waitb(p, ms, &ms.s_full[gg & 1], (gg >> 1) & 1)) return;
+            ptx::tc_fence_after();
+            float s[kN];
+            const uint32_t scol = (gg & 1) ? kColS1 : kColS0;
+            ptx::tmem_ld48(tmem + scol, s);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ms.s_free[gg & 1]);
+
+            const int pos0 = (pc.page_lo + k * kTilePages) * kPage;
+            const int pos = pos0 + i;
+            const bool loaded = (info >> (i / kPage)) & 1u;
+            // value scale of this lane's token; 0 where the slot is not a
+            // cached position (its stored scale may be anything, even NaN)
+            const float kvs = !kFp8 ? 1.f
+                              : (loaded && pos < pc.ctx)
+                                  ? reinterpret_cast<const float *>(smem + C::kScaleOff + stage * C::kScaleBytes)[i]
+                                  : 0.f;
+            const float factor = p.sm_scale_log2 * (kFp8 ? kvs * qscale : 1.f);
+            const float lkvs = kFp8 ? __log2f(kvs) : 0.f;
+            const bool fast = (info & 0xFFu) == 0xFFu && pos0 + kTileM <= min_lim;
+            bool exceed = false;
+#pragma unroll
+            for (int c = 0; c < kN; ++c) {
+                const bool valid = fast || (loaded && pos < ms.col_lim[c]);
+                s[c] = valid ? s[c] * factor : -INFINITY;      // score, log2 units
+                exceed |= s[c] + lkvs > m2[c] + C::kTau;
+            }
+            // all lanes must agree on the stabiliser: vote across the 4 warps
+            const int vote = __any_sync(0xffffffffu, exceed);
+            if (lane == 0) ms.vote[gg & 1][wi] = vote;
+            if (!gsync(p, ms)) return;
+            const bool any = ms.vote[gg & 1][0] | ms.vote[gg & 1][1] | ms.vote[gg & 1][2] | ms.vote[gg & 1][3];
+            if (any) {
+#pragma unroll
+                for (int c = 0; c < kN; ++c) {
+                    const float cm = warp_max(s[c] + lkvs);
+                    if (lane == 0) ms.red[wi][c] = cm;
+                }
+                if (!gsync(p, ms)) return;
+                float alpha[kN];
+                bool moved = false;
+#pragma unroll
+                for (int c = 0; c < kN; ++c) {
+                    const float cm = fmaxf(fmaxf(ms.red[0][c], ms.red[1][c]), fmaxf(ms.red[2][c], ms.red[3][c]));
+                    const float mn = cm > m2[c] + C::kTau ? cm : m2[c];
+                    alpha[c] = mn == m2[c] ? 1.f : exp2f(m2[c] - mn);
+                    moved |= mn != m2[c];
+                    m2[c] = mn;
+                    lsum[c] *= alpha[c];
+                }
+                if (!gsync(p, ms)) return;  // red[] reads done before any reuse
+                if (moved && k > 0) {
+                    // O^T holds earlier tiles: wait for their value MMA, then rescale columns
+                    if (!waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
+                    ptx::tc_fence_after();
+#pragma unroll 1
+                    for (int m = 0; m < 4; ++m) {
+                        float o[kN];
+                        const uint32_t oc = tmem + kColO + 64 * m;
+                        ptx::tmem_ld48(oc, o);
+#pragma unroll
+                        for (int c = 0; c < kN; ++c) o[c] *= alpha[c];
+                        ptx::tmem_st48(oc, o);
+                    }
+                }
+            }
+            // weights: e = exp2(s - m2 + C) enters the row sum; the value MMA
+            // takes e times the token's value scale (FP8) as its P entry.
+            // (s[] is reused to hold the P entry of each row)
+            uint32_t pk[kN / 2];
+#pragma unroll
+            for (int c = 0; c < kN; c += 2) {
+                const float e0 = s[c] == -INFINITY ? 0.f : exp2f(s[c] - m2[c] + C::kC);
+                const float e1 = s[c + 1] == -INFINITY ? 0.f : exp2f(s[c + 1] - m2[c + 1] + C::kC);
+                lsum[c] += e0;
+                lsum[c + 1] += e1;
+                if constexpr (kFp8) {
+                    s[c] = e0 * kvs;
+                    s[c + 1] = e1 * kvs;
+                } else {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(e0, e1);
+                    pk[c / 2] = *reinterpret_cast<uint32_t *>(&h);
+                }
+            }
+            // rows past the context in a loaded page may hold anything; their
+            // weight is 0 but 0 * NaN is NaN, so clear them before the value MMA
+            if (!fast && loaded && pos >= pc.ctx) {
+                unsigned char *stg = smem + C::kKvOff + stage * C::kStageBytes;
+#pragma unroll
+                for (int c = 0; c < C::kVChunks; ++c) {
+                    uint4 *row = reinterpret_cast<uint4 *>(stg + c * C::kChunkBytes + i * 128);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) row[e] = make_uint4(0, 0, 0, 0);
+                }
+            }
+            // the single P buffer is free once the previous tile's value MMA is done
+            if (gg > 0 && !waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
+            unsigned char *pb = smem + C::kPOff;
+            if constexpr (kFp8) {
+                // P = hi + lo, two e4m3 operands (about bf16 precision per weight)
+#pragma unroll
+                for (int j = 0; j < kN / 16; ++j) {
+                    uint4 vh, vl;
+                    uint8_t *bh = reinterpret_cast<uint8_t *>(&vh);
+                    uint8_t *bl = reinterpret_cast<uint8_t *>(&vl);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) split_e4m3(s[16 * j + e], bh[e], bl[e]);
+                    *reinterpret_cast<uint4 *>(pb + j * 2048 + i * 16) = vh;
+                    *reinterpret_cast<uint4 *>(pb + C::kPPart + j * 2048 + i * 16) = vl;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kN / 8; ++j)
+                    *reinterpret_cast<uint4 *>(pb + j * 2048 + i * 16) =
+                        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ms.p_full);
+        }
+        g = g0 + nt;
+
+        // ---- epilogue: row sums, normalised output, log-sum-exp
+        if (!waitb(p, ms, &ms.pv_done, (g - 1) & 1)) return;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kN; ++c) {
+            const float v = warp_sum(lsum[c]);
+            if (lane == 0) ms.red[wi][c] = v;
+        }
+        if (st == 0) {
+#pragma unroll
+            for (int c = 0; c < kN; ++c) ms.m2[c] = m2[c];
+        }
+        if (!gsync(p, ms)) return;
+        if (st < kN) {
+            const float l = ms.red[0][st] + ms.red[1][st] + ms.red[2][st] + ms.red[3][st];
+            const bool bad = piece_bad || ms.col_bad[st];
+            ms.inv_l[st] = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+            ms.lse[st] = bad ? NAN : (l > 0.f ? (ms.m2[st] - C::kC + __log2f(l)) * kLn2 : -INFINITY);
+        }
+        if (!gsync(p, ms)) return;
+#pragma unroll 1
+        for (int m = 0; m < 4; ++m) {
+            float o[kN];
+            const uint32_t oc = tmem + kColO + 64 * m;
+            ptx::tmem_ld48(oc, o);
+            const int d = 128 * m + i;
+            for (int c = 0; c < rows_here; ++c) {
+                const float v = o[c] * ms.inv_l[c];
+                const int64_t r = r0 + c;
+                if (pc.single)
+                    store_out(p.out, ((int64_t)pc.b * p.R + r) * kDl + d, v, p.out_f32);
+                else
+                    p.part_o[((int64_t)pc.piece * p.R + r) * kDl + d] = v;
+            }
+        }
+        if (st < rows_here) {
+            const int64_t r = r0 + st;
+            if (pc.single) {
+                if (p.lse) p.lse[(int64_t)pc.b * p.R + r] = ms.lse[st];
+            } else {
+                p.part_lse[(int64_t)pc.piece * p.R + r] = ms.lse[st];
+            }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&ms.o_free);
+        if (!gsync(p, ms)) return;  // smem per-piece state reused next piece
+        ++pi;
+    });
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_decode_kernel(const __grid_constant__ Problem p, const __grid_constant__ CUtensorMap map_a,
+                     const __grid_constant__ CUtensorMap map_b) {
+    using C = Cfg<kFp8>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Misc &ms = *reinterpret_cast<Misc *>(smem + C::kMiscOff);
+    const int warp = threadIdx.x >> 5;
+    const int slot = blockIdx.x / p.n_groups;
+    const int g_idx = blockIdx.x % p.n_groups;
+
+    // Zero the KV stages once: rows never loaded then hold finite values.
+    for (int o = threadIdx.x * 16; o < C::kStages * C::kStageBytes; o += kThreads * 16)
+        *reinterpret_cast<uint4 *>(smem + C::kKvOff + o) = make_uint4(0, 0, 0, 0);
+    ptx::fence_proxy_async_smem();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&ms.kv_full[s], 1);
+            ptx::mbar_init(&ms.kv_empty[s], 1);
+            ptx::mbar_init(&ms.s_full[s], 1);
+            ptx::mbar_init(&ms.s_free[s], 4);
+        }
+        ptx::mbar_init(&ms.p_full, 4);
+        ptx::mbar_init(&ms.pv_done, 1);
+        ptx::mbar_init(&ms.q_ready, 4);
+        ptx::mbar_init(&ms.o_free, 4);
+        ptx::mbar_init(&ms.drain, 1);
+        ptx::mbar_init(&ms.group, 4);
+        ms.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && threadIdx.x == 0) {
+        ptx::prefetch_tensormap(&map_a);
+        if (kFp8) ptx::prefetch_tensormap(&map_b);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&ms.tmem_base, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+
+    if (warp == 0)
+        producer<kFp8>(p, &map_a, &map_b, smem, ms, slot);
+    else if (warp == 1)
+        mma_issuer<kFp8>(p, smem, ms, slot);
+    else
+        softmax_role<kFp8>(p, smem, ms, slot, g_idx);
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(ms.tmem_base, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D view of the page pool: [num_pages*16 rows][576 elements], boxes of 16 rows.
+bool make_kv_map(CUtensorMap *map, const void *base, int num_pages, bool fp8, uint32_t box_cols,
+                 CUtensorMapSwizzle swz) {
+    auto encode = get_encode_fn();
+    if (!encode) return false;
+    const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)num_pages * kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * (fp8 ? 1 : 2)};
+    const cuuint32_t box[2] = {box_cols, (cuuint32_t)kPage};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool kFp8>
+int launch_impl(const Problem &p, cudaStream_t stream) {
+    CUtensorMap ma, mb;
+    bool ok;
+    if (kFp8) {
+        ok = make_kv_map(&ma, p.kv, p.num_pages, true, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_kv_map(&mb, p.kv, p.num_pages, true, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+    } else {
+        ok = make_kv_map(&ma, p.kv, p.num_pages, false, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+        mb = ma;
+    }
+    if (!ok) return MLA_ERR_CUDA;
+    const int smem = smem_bytes<kFp8>();
+    cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) {
+        tc_decode_kernel<kFp8><<<p.n_slots * p.n_groups, kThreads, smem, stream>>>(p, ma, mb);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+static_assert(smem_bytes<true>() <= 232448, "FP8 tile does not fit shared memory");
+static_assert(smem_bytes<false>() <= 232448, "bf16 tile does not fit shared memory");
+
+}  // namespace
+
+int tc_rows_per_group() { return kN; }
+
+int launch_tc(const Problem &p, cudaStream_t stream) {
+    if (p.rows_per_group != kN) return MLA_ERR_INVALID_ARG;
+    return p.kv_scale ? launch_impl<true>(p, stream) : launch_impl<false>(p, stream);
+}
+
 }  // namespace mla
