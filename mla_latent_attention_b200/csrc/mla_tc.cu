@@ -26,14 +26,14 @@
 //     as stored and never dequantised.
 // bf16 caches use kind::f16 MMAs with bf16 P.
 //
-// Warp roles (192 threads): warp 0 issues TMA page loads, warp 1 issues the
-// MMAs and owns tensor memory, warps 2-5 (one per TMEM lane quadrant) run the
-// online softmax and the epilogue; thread (warp w, lane l) owns tile position
-// / TMEM lane 32*(w%4) + l.
+// Warp roles (320 threads): warp 0 issues TMA page loads, warp 1 issues the
+// MMAs and owns tensor memory, warps 2-9 run the online softmax and the
+// epilogue.  Thread (warp w, lane l) owns tile position / TMEM lane
+// 32*(w%4) + l; warps 2-5 take query columns 0-23 and warps 6-9 columns 24-47.
 //
 // Softmax stabiliser: per query row a running bound m2 on the log2 weight
 // u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
-// all lanes.  It moves only when some weight exceeds it by more than TAU
+// all lanes of a column half.  It moves only when some weight exceeds it by more than TAU
 // (then O^T and the row sums are rescaled), which after the first tile is
 // rare.  Weights are exp2(u - m2 + C), at most 2^(TAU+C), chosen to stay in
 // the e4m3 range for FP8.  Row sums are kept per lane and reduced once per
@@ -55,8 +55,9 @@ namespace {
 constexpr int kN = 48;            // query rows per CTA (MMA N)
 constexpr int kTileM = 128;       // positions per tile (MMA M)
 constexpr int kTilePages = kTileM / kPage;
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kSoftmaxThreads = 256;
+constexpr int kHalf = 24;              // query columns per softmax thread (two halves of 48)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;  // O block m at kColO + 64m
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -90,16 +91,18 @@ struct Cfg {
 struct Misc {
     uint64_t kv_full[2], kv_empty[2], s_full[2], s_free[2];
     uint64_t p_full, pv_done, q_ready, o_free, drain;
-    uint64_t group;           // barrier of the four softmax warps (bounded, unlike bar.sync)
+    uint64_t all_sync;        // the eight softmax warps (bounded waits, unlike bar.sync)
+    uint64_t half_sync[2];    // the four softmax warps of each column half
     uint32_t tmem_base;
     int abort;
     uint32_t stage_info[2];   // bit i: page slot i loaded; bit 31: a page of the tile was invalid
-    int vote[2][4];
+    int vote[2][2][4];        // [half][tile parity][warp]
     int col_lim[kN];          // positions visible to column r within this piece, 0 = none
     int col_bad[kN];
     float qscale;
-    float red[4][kN];
-    float m2[kN];
+    float amax[8];
+    float red[2][4][kHalf];   // [half][warp][column]
+    float m2c[kN];
     float inv_l[kN];
     float lse[kN];
 };
@@ -121,14 +124,17 @@ __device__ __forceinline__ bool waitb(const Problem &p, Misc &ms, uint64_t *bar,
     return false;
 }
 
-// Barrier of the four softmax warps.  An mbarrier with a bounded wait: if a
-// warp has stopped on a timeout, the others give up too instead of hanging.
+// Barrier of a group of softmax warps: an mbarrier counting one arrival per
+// warp, with a bounded wait, so that if a warp has stopped on a timeout the
+// others give up too instead of hanging.
 struct GroupSync {
-    uint32_t phase = 0;
+    uint64_t *bar;
+    uint32_t phase;
+    __device__ explicit GroupSync(uint64_t *b) : bar(b), phase(0) {}
     __device__ __forceinline__ bool operator()(const Problem &p, Misc &ms) {
         __syncwarp();
-        if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&ms.group);
-        const bool ok = waitb(p, ms, &ms.group, phase & 1);
+        if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
+        const bool ok = waitb(p, ms, bar, phase & 1);
         ++phase;
         return ok;
     }
@@ -376,10 +382,10 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
             }
         }
         amax = warp_max(amax);
-        const int w = (threadIdx.x >> 5) - 2;
-        if ((threadIdx.x & 31) == 0) ms.red[w][0] = amax;
+        if ((threadIdx.x & 31) == 0) ms.amax[(threadIdx.x >> 5) - 2] = amax;
         if (!gsync(p, ms)) return false;
-        amax = fmaxf(fmaxf(ms.red[0][0], ms.red[1][0]), fmaxf(ms.red[2][0], ms.red[3][0]));
+#pragma unroll
+        for (int w = 0; w < 8; ++w) amax = fmaxf(amax, ms.amax[w]);
         // A power-of-two scale keeps q/s a bf16 value, which hi + lo then
         // represents exactly (short of e4m3 underflow far below the largest q).
         int e2 = 0;
@@ -440,14 +446,19 @@ template <bool kFp8>
 __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, int slot, int g_idx) {
     using C = Cfg<kFp8>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int w8 = warp - 2;                   // 0..7
+    const int h = w8 >> 2;                     // column half: columns [24h, 24h + 24)
+    const int w4 = w8 & 3;                     // warp within the half
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int i = quad * 32 + lane;            // tile position / TMEM lane
-    const int st = threadIdx.x - 64;           // 0..127 for cooperative loops
-    const int wi = warp - 2;                   // 0..3 slot in reduction buffers
+    const int st = threadIdx.x - 64;           // 0..255 for cooperative loops
+    const int hst = w4 * 32 + lane;            // 0..127 within the half
+    const int cb = h * kHalf;
     const uint32_t tmem = ms.tmem_base + ((uint32_t)(quad * 32) << 16);
     const int r0 = g_idx * kN;
-    uint32_t g = 0, pi = 0;
-    GroupSync gsync;
+    constexpr float kEmpty = -1e30f;           // stabiliser of a column that has seen nothing yet
+    uint32_t g = 0;
+    GroupSync all_sync(&ms.all_sync), hsync(&ms.half_sync[h]);
 
     for_each_piece(p, slot, [&](const Piece &pc) {
         if (aborted(ms)) return;
@@ -462,7 +473,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 const int v = visible(p, pc.b, r / p.H, pc.ctx);
                 if (v < 0) {
                     bad = 1;
-                    if (r % p.H == 0 || st == 0) report_error(p.err, MLA_DEV_BAD_VIS, pc.b * p.T + r / p.H);
+                    report_error(p.err, MLA_DEV_BAD_VIS, pc.b * p.T + r / p.H);
                 } else {
                     lim = min(v, pc.page_hi * kPage);
                 }
@@ -471,10 +482,10 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             ms.col_bad[st] = bad;
         }
         if (st == 0 && pc.bad_ctx && g_idx == 0) report_error(p.err, MLA_DEV_BAD_CTX, pc.b);
-        if (!gsync(p, ms)) return;
+        if (!all_sync(p, ms)) return;
         const int rows_here = min(kN, p.R - r0);
-        int min_lim = INT_MAX;
-        for (int c = 0; c < rows_here; ++c) min_lim = min(min_lim, ms.col_lim[c]);
+        int min_lim = INT_MAX;  // over this half's real columns
+        for (int c = cb; c < min(cb + kHalf, rows_here); ++c) min_lim = min(min_lim, ms.col_lim[c]);
 
         if (nt == 0) {  // nothing to read: write the empty (or invalid) result
             for (int e = st; e < rows_here * kDl; e += kSoftmaxThreads) {
@@ -483,21 +494,22 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 store_out(p.out, ((int64_t)pc.b * p.R + r0 + c) * kDl + d, bad ? NAN : 0.f, p.out_f32);
                 if (d == 0 && p.lse) p.lse[(int64_t)pc.b * p.R + r0 + c] = bad ? NAN : -INFINITY;
             }
-            gsync(p, ms);
+            all_sync(p, ms);
             return;
         }
 
-        if (!load_query<kFp8>(p, smem, ms, pc.b, r0, st, gsync)) return;
+        if (!load_query<kFp8>(p, smem, ms, pc.b, r0, st, all_sync)) return;
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ms.q_ready);
-        if (!gsync(p, ms)) return;  // qscale visible
+        if (!all_sync(p, ms)) return;  // qscale visible
         const float qscale = kFp8 ? ms.qscale : 1.f;
 
-        float m2[kN], lsum[kN];
+        // m2c = stabiliser - C: weights are ex2(score - m2c)
+        float m2c[kHalf], lsum[kHalf];
 #pragma unroll
-        for (int c = 0; c < kN; ++c) {
-            m2[c] = -INFINITY;
+        for (int c = 0; c < kHalf; ++c) {
+            m2c[c] = kEmpty;
             lsum[c] = 0.f;
         }
         bool piece_bad = false;
@@ -510,9 +522,8 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             piece_bad |= (info >> 31) != 0;
             if (!waitb(p, ms, &ms.s_full[gg & 1], (gg >> 1) & 1)) return;
             ptx::tc_fence_after();
-            float s[kN];
-            const uint32_t scol = (gg & 1) ? kColS1 : kColS0;
-            ptx::tmem_ld48(tmem + scol, s);
+            float s[kHalf];
+            ptx::tmem_ld24(tmem + ((gg & 1) ? kColS1 : kColS0) + cb, s);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&ms.s_free[gg & 1]);
@@ -529,73 +540,67 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             const float factor = p.sm_scale_log2 * (kFp8 ? kvs * qscale : 1.f);
             const float lkvs = kFp8 ? __log2f(kvs) : 0.f;
             const bool fast = (info & 0xFFu) == 0xFFu && pos0 + kTileM <= min_lim;
+            // u = s + lkvs exceeds the stabiliser by more than TAU iff s > m2c + (C + TAU - lkvs)
+            const float kx = C::kC + C::kTau - lkvs;
             bool exceed = false;
 #pragma unroll
-            for (int c = 0; c < kN; ++c) {
-                const bool valid = fast || (loaded && pos < ms.col_lim[c]);
-                s[c] = valid ? s[c] * factor : -INFINITY;      // score, log2 units
-                exceed |= s[c] + lkvs > m2[c] + C::kTau;
+            for (int c = 0; c < kHalf; ++c) {
+                const bool valid = fast || (loaded && pos < ms.col_lim[cb + c]);
+                s[c] = valid ? s[c] * factor : -INFINITY;       // score, log2 units
+                exceed |= s[c] > m2c[c] + kx;
             }
-            // all lanes must agree on the stabiliser: vote across the 4 warps
+            // all lanes of the half must agree on the stabiliser
             const int vote = __any_sync(0xffffffffu, exceed);
-            if (lane == 0) ms.vote[gg & 1][wi] = vote;
-            if (!gsync(p, ms)) return;
-            const bool any = ms.vote[gg & 1][0] | ms.vote[gg & 1][1] | ms.vote[gg & 1][2] | ms.vote[gg & 1][3];
-            if (any) {
+            if (lane == 0) ms.vote[h][gg & 1][w4] = vote;
+            if (!hsync(p, ms)) return;
+            const int *vv = ms.vote[h][gg & 1];
+            if (vv[0] | vv[1] | vv[2] | vv[3]) {
 #pragma unroll
-                for (int c = 0; c < kN; ++c) {
+                for (int c = 0; c < kHalf; ++c) {
                     const float cm = warp_max(s[c] + lkvs);
-                    if (lane == 0) ms.red[wi][c] = cm;
+                    if (lane == 0) ms.red[h][w4][c] = cm;
                 }
-                if (!gsync(p, ms)) return;
-                float alpha[kN];
+                if (!hsync(p, ms)) return;
+                float alpha[kHalf];
                 bool moved = false;
 #pragma unroll
-                for (int c = 0; c < kN; ++c) {
-                    const float cm = fmaxf(fmaxf(ms.red[0][c], ms.red[1][c]), fmaxf(ms.red[2][c], ms.red[3][c]));
-                    const float mn = cm > m2[c] + C::kTau ? cm : m2[c];
-                    alpha[c] = mn == m2[c] ? 1.f : exp2f(m2[c] - mn);
-                    moved |= mn != m2[c];
-                    m2[c] = mn;
+                for (int c = 0; c < kHalf; ++c) {
+                    const float cm = fmaxf(fmaxf(ms.red[h][0][c], ms.red[h][1][c]),
+                                           fmaxf(ms.red[h][2][c], ms.red[h][3][c]));
+                    const float old = m2c[c] + C::kC;
+                    const float mn = cm > old + C::kTau ? cm : old;
+                    alpha[c] = mn == old ? 1.f : ptx::ex2(old - mn);
+                    moved |= mn != old;
+                    m2c[c] = mn - C::kC;
                     lsum[c] *= alpha[c];
                 }
-                if (!gsync(p, ms)) return;  // red[] reads done before any reuse
+                if (!hsync(p, ms)) return;  // red[] reads done before any reuse
                 if (moved && k > 0) {
                     // O^T holds earlier tiles: wait for their value MMA, then rescale columns
                     if (!waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
                     ptx::tc_fence_after();
 #pragma unroll 1
                     for (int m = 0; m < 4; ++m) {
-                        float o[kN];
-                        const uint32_t oc = tmem + kColO + 64 * m;
-                        ptx::tmem_ld48(oc, o);
+                        float o[kHalf];
+                        const uint32_t oc = tmem + kColO + 64 * m + cb;
+                        ptx::tmem_ld24(oc, o);
 #pragma unroll
-                        for (int c = 0; c < kN; ++c) o[c] *= alpha[c];
-                        ptx::tmem_st48(oc, o);
+                        for (int c = 0; c < kHalf; ++c) o[c] *= alpha[c];
+                        ptx::tmem_st24(oc, o);
                     }
                 }
             }
-            // weights: e = exp2(s - m2 + C) enters the row sum; the value MMA
-            // takes e times the token's value scale (FP8) as its P entry.
-            // (s[] is reused to hold the P entry of each row)
-            uint32_t pk[kN / 2];
+            // weights e = ex2(s - m2c) enter the row sums; the value MMA takes
+            // e times the token's value scale (FP8) as its P entry
 #pragma unroll
-            for (int c = 0; c < kN; c += 2) {
-                const float e0 = s[c] == -INFINITY ? 0.f : exp2f(s[c] - m2[c] + C::kC);
-                const float e1 = s[c + 1] == -INFINITY ? 0.f : exp2f(s[c + 1] - m2[c + 1] + C::kC);
-                lsum[c] += e0;
-                lsum[c + 1] += e1;
-                if constexpr (kFp8) {
-                    s[c] = e0 * kvs;
-                    s[c + 1] = e1 * kvs;
-                } else {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(e0, e1);
-                    pk[c / 2] = *reinterpret_cast<uint32_t *>(&h);
-                }
+            for (int c = 0; c < kHalf; ++c) {
+                const float e = ptx::ex2(s[c] - m2c[c]);
+                lsum[c] += e;
+                s[c] = kFp8 ? e * kvs : e;
             }
             // rows past the context in a loaded page may hold anything; their
             // weight is 0 but 0 * NaN is NaN, so clear them before the value MMA
-            if (!fast && loaded && pos >= pc.ctx) {
+            if (h == 0 && !fast && loaded && pos >= pc.ctx) {
                 unsigned char *stg = smem + C::kKvOff + stage * C::kStageBytes;
 #pragma unroll
                 for (int c = 0; c < C::kVChunks; ++c) {
@@ -608,22 +613,47 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             if (gg > 0 && !waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
             unsigned char *pb = smem + C::kPOff;
             if constexpr (kFp8) {
-                // P = hi + lo, two e4m3 operands (about bf16 precision per weight)
+                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of the half
+                uint32_t hw[kHalf / 4], lw[kHalf / 4];
 #pragma unroll
-                for (int j = 0; j < kN / 16; ++j) {
-                    uint4 vh, vl;
-                    uint8_t *bh = reinterpret_cast<uint8_t *>(&vh);
-                    uint8_t *bl = reinterpret_cast<uint8_t *>(&vl);
+                for (int w = 0; w < kHalf / 4; ++w) {
+                    uint32_t hp[2], lp[2];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) split_e4m3(s[16 * j + e], bh[e], bl[e]);
-                    *reinterpret_cast<uint4 *>(pb + j * 2048 + i * 16) = vh;
-                    *reinterpret_cast<uint4 *>(pb + C::kPPart + j * 2048 + i * 16) = vl;
+                    for (int q = 0; q < 2; ++q) {
+                        const float a = s[4 * w + 2 * q], b = s[4 * w + 2 * q + 1];
+                        hp[q] = ptx::e4m3x2(a, b);
+                        float fa, fb;
+                        ptx::e4m3x2_to_f32(hp[q], &fa, &fb);
+                        lp[q] = ptx::e4m3x2(a - fa, b - fb);
+                    }
+                    hw[w] = hp[0] | (hp[1] << 16);
+                    lw[w] = lp[0] | (lp[1] << 16);
+                }
+                // 16-row groups: half 0 owns group 0 and the low 8 bytes of group 1,
+                // half 1 the high 8 bytes of group 1 and group 2
+                unsigned char *g16 = pb + (h == 0 ? 0 : 4096) + i * 16;
+                unsigned char *g8 = pb + 2048 + i * 16 + (h == 0 ? 0 : 8);
+                const int w16 = h == 0 ? 0 : 2, w8o = h == 0 ? 4 : 0;
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t *src = part ? lw : hw;
+                    const int off = part ? C::kPPart : 0;
+                    *reinterpret_cast<uint4 *>(g16 + off) =
+                        make_uint4(src[w16], src[w16 + 1], src[w16 + 2], src[w16 + 3]);
+                    *reinterpret_cast<uint2 *>(g8 + off) = make_uint2(src[w8o], src[w8o + 1]);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < kN / 8; ++j)
-                    *reinterpret_cast<uint4 *>(pb + j * 2048 + i * 16) =
-                        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                for (int j = 0; j < 3; ++j) {
+                    uint32_t wv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(s[8 * j + 2 * q], s[8 * j + 2 * q + 1]);
+                        wv[q] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    *reinterpret_cast<uint4 *>(pb + (3 * h + j) * 2048 + i * 16) =
+                        make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
@@ -636,50 +666,51 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (!waitb(p, ms, &ms.pv_done, (g - 1) & 1)) return;
         ptx::tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kN; ++c) {
+        for (int c = 0; c < kHalf; ++c) {
             const float v = warp_sum(lsum[c]);
-            if (lane == 0) ms.red[wi][c] = v;
+            if (lane == 0) ms.red[h][w4][c] = v;
         }
-        if (st == 0) {
+        if (hst == 0) {
 #pragma unroll
-            for (int c = 0; c < kN; ++c) ms.m2[c] = m2[c];
+            for (int c = 0; c < kHalf; ++c) ms.m2c[cb + c] = m2c[c];
         }
-        if (!gsync(p, ms)) return;
-        if (st < kN) {
-            const float l = ms.red[0][st] + ms.red[1][st] + ms.red[2][st] + ms.red[3][st];
-            const bool bad = piece_bad || ms.col_bad[st];
-            ms.inv_l[st] = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
-            ms.lse[st] = bad ? NAN : (l > 0.f ? (ms.m2[st] - C::kC + __log2f(l)) * kLn2 : -INFINITY);
+        if (!hsync(p, ms)) return;
+        if (hst < kHalf) {
+            const int col = cb + hst;
+            const float l = ms.red[h][0][hst] + ms.red[h][1][hst] + ms.red[h][2][hst] + ms.red[h][3][hst];
+            const bool bad = piece_bad || ms.col_bad[col];
+            // ln sum_j exp(score_j) = (m2c + log2 l) * ln 2
+            ms.inv_l[col] = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+            ms.lse[col] = bad ? NAN : (l > 0.f ? (ms.m2c[col] + __log2f(l)) * kLn2 : -INFINITY);
         }
-        if (!gsync(p, ms)) return;
+        if (!hsync(p, ms)) return;
+        const int ncols = min(kHalf, rows_here - cb);
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
-            float o[kN];
-            const uint32_t oc = tmem + kColO + 64 * m;
-            ptx::tmem_ld48(oc, o);
+            float o[kHalf];
+            ptx::tmem_ld24(tmem + kColO + 64 * m + cb, o);
             const int d = 128 * m + i;
-            for (int c = 0; c < rows_here; ++c) {
-                const float v = o[c] * ms.inv_l[c];
-                const int64_t r = r0 + c;
+            for (int c = 0; c < ncols; ++c) {
+                const float v = o[c] * ms.inv_l[cb + c];
+                const int64_t r = r0 + cb + c;
                 if (pc.single)
                     store_out(p.out, ((int64_t)pc.b * p.R + r) * kDl + d, v, p.out_f32);
                 else
                     p.part_o[((int64_t)pc.piece * p.R + r) * kDl + d] = v;
             }
         }
-        if (st < rows_here) {
-            const int64_t r = r0 + st;
+        if (hst < ncols) {
+            const int64_t r = r0 + cb + hst;
             if (pc.single) {
-                if (p.lse) p.lse[(int64_t)pc.b * p.R + r] = ms.lse[st];
+                if (p.lse) p.lse[(int64_t)pc.b * p.R + r] = ms.lse[cb + hst];
             } else {
-                p.part_lse[(int64_t)pc.piece * p.R + r] = ms.lse[st];
+                p.part_lse[(int64_t)pc.piece * p.R + r] = ms.lse[cb + hst];
             }
         }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ms.o_free);
-        if (!gsync(p, ms)) return;  // smem per-piece state reused next piece
-        ++pi;
+        all_sync(p, ms);  // smem per-piece state reused next piece
     });
 }
 
@@ -705,14 +736,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&ms.kv_full[s], 1);
             ptx::mbar_init(&ms.kv_empty[s], 1);
             ptx::mbar_init(&ms.s_full[s], 1);
-            ptx::mbar_init(&ms.s_free[s], 4);
+            ptx::mbar_init(&ms.s_free[s], 8);
+            ptx::mbar_init(&ms.half_sync[s], 4);
         }
-        ptx::mbar_init(&ms.p_full, 4);
+        ptx::mbar_init(&ms.p_full, 8);
         ptx::mbar_init(&ms.pv_done, 1);
-        ptx::mbar_init(&ms.q_ready, 4);
-        ptx::mbar_init(&ms.o_free, 4);
+        ptx::mbar_init(&ms.q_ready, 8);
+        ptx::mbar_init(&ms.o_free, 8);
         ptx::mbar_init(&ms.drain, 1);
-        ptx::mbar_init(&ms.group, 4);
+        ptx::mbar_init(&ms.all_sync, 8);
         ms.abort = 0;
         ptx::fence_mbar_init();
     }
