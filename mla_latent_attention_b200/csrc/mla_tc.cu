@@ -7,36 +7,37 @@
 // 128 cached positions (8 pages of 16).
 //
 // Orientation ("swap AB"): positions are the MMA M dimension (128 TMEM lanes)
-// and query rows the N dimension (48 columns), so
-//     S^T [128 x 48] = KV_tile[128 x 576] . Q^T          (scores)
-//     O^T [512 x 48] += V_tile^T[512 x 128] . P^T         (values, 4 blocks of 128)
-// S^T (two buffers) and O^T live in tensor memory: 2*48 + 4*48 columns of
-// the 512.  With the rows as M instead, a 128 x 512 fp32 O alone would fill
-// all of tensor memory.
+// and query rows the N dimension, so
+//     S^T [128 x N] = KV_tile[128 x 576] . Q^T           (scores)
+//     O^T [512 x N] += V_tile^T[512 x 128] . P^T          (values, 4 blocks of 128)
+// and both accumulators live in tensor memory.  With the rows as M instead, a
+// 128 x 512 fp32 O alone would fill all of tensor memory.
 //
 // FP8 caches are consumed as stored, by kind::f8f6f4 MMAs:
 //   * scores: the query is split on chip into two e4m3 parts, hi = e4m3(q/s)
-//     and lo = e4m3(q/s - hi), with one power-of-two scale s per CTA, and S
-//     accumulates K.hi + K.lo.  For a bf16 query hi + lo is exact (a bf16
-//     significand has 8 bits, hi takes the top 4 and the remainder fits lo),
-//     at the tensor-core cost of one bf16 MMA; the per-token scale multiplies
-//     S^T lane by lane.
-//   * values: P^T is split the same way into two e4m3 operands, after the
-//     per-token value scale has been folded into each weight, so V is read
-//     as stored and never dequantised.
-// bf16 caches use kind::f16 MMAs with bf16 P.
+//     and lo = e4m3(q/s - hi), with one power-of-two scale s per CTA.  For a
+//     bf16 query hi + lo is exact (a bf16 significand has 8 bits, hi takes
+//     the top 4 and the remainder fits lo).  hi and lo are stacked along N, so
+//     one N = 96 MMA per K step yields both partial scores (the KV tile is
+//     read once) and the softmax adds the two halves.  The per-token scale
+//     multiplies S^T lane by lane.
+//   * values: the weights, with the per-token value scale folded in, are
+//     split the same way into hi and lo, stacked along N = 96; the epilogue
+//     adds the two halves of O^T.  V is read as stored, never dequantised.
+// bf16 caches use kind::f16 MMAs with N = 48 and bf16 P.
 //
-// Warp roles (320 threads): warp 0 issues TMA page loads, warp 1 issues the
-// MMAs and owns tensor memory, warps 2-9 run the online softmax and the
-// epilogue.  Thread (warp w, lane l) owns tile position / TMEM lane
-// 32*(w%4) + l; warps 2-5 take query columns 0-23 and warps 6-9 columns 24-47.
+// Warp roles (320 threads): warp 0 issues TMA page loads (and warms L2 with
+// the tiles after them), warp 1 issues the MMAs -- each as soon as its
+// operands are ready -- and owns tensor memory, warps 2-9 run the online
+// softmax and the epilogue.  Thread (warp w, lane l) owns tile position /
+// TMEM lane 32*(w%4) + l; warps 2-5 take query rows 0-23, warps 6-9 rows 24-47.
 //
 // Softmax stabiliser: per query row a running bound m2 on the log2 weight
 // u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
-// all lanes of a column half.  It moves only when some weight exceeds it by more than TAU
-// (then O^T and the row sums are rescaled), which after the first tile is
-// rare.  Weights are exp2(u - m2 + C), at most 2^(TAU+C), chosen to stay in
-// the e4m3 range for FP8.  Row sums are kept per lane and reduced once per
+// the lanes of a row half.  It moves only when some weight exceeds it by more
+// than TAU (then O^T and the row sums are rescaled), which after the first
+// tile is rare.  Weights are exp2(u - m2 + C), at most 2^(TAU+C), which keeps
+// the e4m3 weights in range.  Row sums are kept per lane and reduced once per
 // piece.
 //
 // Every wait is bounded: after two seconds the CTA records a timeout in the
@@ -52,21 +53,27 @@
 namespace mla {
 namespace {
 
-constexpr int kN = 48;            // query rows per CTA (MMA N)
-constexpr int kTileM = 128;       // positions per tile (MMA M)
+constexpr int kN = 48;                 // query rows per CTA
+constexpr int kTileM = 128;            // positions per tile (MMA M)
 constexpr int kTilePages = kTileM / kPage;
 constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr int kSoftmaxThreads = 256;
-constexpr int kHalf = 24;              // query columns per softmax thread (two halves of 48)
+constexpr int kHalf = 24;              // query rows per softmax thread (two halves of 48)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;  // O block m at kColO + 64m
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kDevTimeout = 4;
+constexpr int kPrefetchAhead = 3;      // L2 prefetch distance, tiles
 
 template <bool kFp8>
 struct Cfg {
-    static constexpr int kStages = kFp8 ? 2 : 1;
-    // KV stage: chunks of [128 positions][128 B], plus for FP8 the RoPE chunk [128][64 B]
+    static constexpr int kStages = kFp8 ? 2 : 1;                                   // KV stages
+    static constexpr int kSBufs = kFp8 ? 1 : 2;                                    // S^T buffers
+    static constexpr int kNMma = kFp8 ? 2 * kN : kN;                               // MMA N (hi|lo stacked)
+    // tensor memory columns
+    static constexpr uint32_t kColS1 = 64;                                         // second S^T buffer
+    static constexpr uint32_t kColO = 128;
+    static constexpr uint32_t kOStride = kFp8 ? 96u : 64u;                         // O block m at kColO + m*stride
+    // KV stage: chunks of [128 positions][128 B]; FP8 adds the RoPE chunk [128][64 B]
     static constexpr int kChunkBytes = kTileM * 128;                              // 16384
     static constexpr int kVChunks = kFp8 ? 4 : 8;                                 // chunks holding c_kv
     static constexpr int kStageBytes = kFp8 ? 4 * kChunkBytes + kTileM * 64 : 9 * kChunkBytes;
@@ -74,34 +81,36 @@ struct Cfg {
     static constexpr int kScaleOff = kKvOff + kStages * kStageBytes;               // FP8: 512 B / stage
     static constexpr int kScaleBytes = kFp8 ? kTileM * 4 : 0;
     static constexpr int kQOff = (kScaleOff + kStages * kScaleBytes + 1023) & ~1023;
-    static constexpr int kQChunk = kN * 128;                                       // 6144
-    static constexpr int kQPart = kFp8 ? 4 * kQChunk + kN * 64 : 9 * kQChunk;      // one operand
-    static constexpr int kQBytes = kFp8 ? 2 * kQPart : kQPart;
+    // Q (MMA B operand, K-major): FP8 chunk c = [96 rows: hi 0-47, lo 48-95][128 B]; bf16 [48][128 B]
+    static constexpr int kQChunk = kNMma * 128;                                    // 12288 / 6144
+    static constexpr int kQRopeOff = 4 * kQChunk;                                  // FP8 RoPE chunk [96][64 B]
+    static constexpr int kQBytes = kFp8 ? 4 * kQChunk + kNMma * 64 : 9 * kQChunk;
     static constexpr int kPOff = (kQOff + kQBytes + 1023) & ~1023;
-    static constexpr int kPGroupRows = kFp8 ? 16 : 8;                              // rows per 16 B
-    static constexpr int kPPart = (kN / kPGroupRows) * kTileM * 16;                // one P operand
-    static constexpr int kPBytes = kFp8 ? 2 * kPPart : kPPart;                     // FP8: hi and lo
+    // P^T (MMA B operand, MN-major, no swizzle): groups of 16 B of rows x 128 positions
+    static constexpr int kPGroupRows = kFp8 ? 16 : 8;
+    static constexpr int kPBytes = (kNMma / kPGroupRows) * kTileM * 16;           // 12288 both
+    static constexpr int kPLoOff = kFp8 ? (kN / 16) * kTileM * 16 : 0;             // lo rows start (group 3)
     static constexpr int kMiscOff = kPOff + kPBytes;
     static constexpr int kPageBytes = kFp8 ? (4 * 2048 + 1024 + 64) : 9 * 2048;   // bytes a page brings
     // exponent offset C and lazy threshold TAU of the softmax stabiliser
-    static constexpr float kC = kFp8 ? 6.5f : 0.f;
-    static constexpr float kTau = kFp8 ? 2.f : 8.f;
+    static constexpr float kC = kFp8 ? 4.5f : 0.f;
+    static constexpr float kTau = kFp8 ? 4.f : 8.f;
 };
 
 struct Misc {
     uint64_t kv_full[2], kv_empty[2], s_full[2], s_free[2];
     uint64_t p_full, pv_done, q_ready, o_free, drain;
     uint64_t all_sync;        // the eight softmax warps (bounded waits, unlike bar.sync)
-    uint64_t half_sync[2];    // the four softmax warps of each column half
+    uint64_t half_sync[2];    // the four softmax warps of each row half
     uint32_t tmem_base;
     int abort;
     uint32_t stage_info[2];   // bit i: page slot i loaded; bit 31: a page of the tile was invalid
     int vote[2][2][4];        // [half][tile parity][warp]
-    int col_lim[kN];          // positions visible to column r within this piece, 0 = none
+    int col_lim[kN];          // positions visible to row r within this piece, 0 = none
     int col_bad[kN];
     float qscale;
     float amax[8];
-    float red[2][4][kHalf];   // [half][warp][column]
+    float red[2][4][kHalf];   // [half][warp][row]
     float m2c[kN];
     float inv_l[kN];
     float lse[kN];
@@ -156,8 +165,7 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Query split for the e4m3 score MMA: hi = e4m3(x), lo = e4m3(x - hi), so that
-// hi + lo carries about twice the mantissa bits of one e4m3 value.
+// Query split for the e4m3 score MMA: hi = e4m3(x), lo = e4m3(x - hi).
 __device__ __forceinline__ void split_e4m3(float x, uint8_t &hi, uint8_t &lo) {
     const __nv_fp8_e4m3 h(x);              // round to nearest, saturating
     const __nv_fp8_e4m3 l(x - float(h));
@@ -174,8 +182,27 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
     using C = Cfg<kFp8>;
     const int lane = threadIdx.x & 31;
     uint32_t g = 0;
+    // L2 warm-up of tile k of a piece: page ids, then one prefetch per page/box
+    auto prefetch_tile = [&](const Piece &pc, int k) {
+        const int pg0 = pc.page_lo + k * kTilePages;
+        const int npg = min(kTilePages, pc.page_hi - pg0);
+        if (npg <= 0 || lane >= npg) return;
+        const int pid = __ldg(p.page_table + (int64_t)pc.b * p.pt_stride + pg0 + lane);
+        if (pid < 0 || pid >= p.num_pages) return;
+        const int y = pid * kPage;
+        if constexpr (kFp8) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ptx::tma_prefetch_2d(map_a, 128 * c, y);
+            ptx::tma_prefetch_2d(map_b, 512, y);
+            ptx::bulk_prefetch(p.kv_scale + (int64_t)pid * kPage, 64);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 9; ++c) ptx::tma_prefetch_2d(map_a, 64 * c, y);
+        }
+    };
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
+        for (int k = 1; k < min(nt, kPrefetchAhead); ++k) prefetch_tile(pc, k);
         for (int k = 0; k < nt; ++k, ++g) {
             if (aborted(ms)) return;
             const int stage = g % C::kStages;
@@ -214,6 +241,7 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                                          64 * c, y);
                 }
             }
+            if (k + kPrefetchAhead < nt) prefetch_tile(pc, k + kPrefetchAhead);
         }
     });
     // make sure no copy is still landing when the CTA leaves
@@ -232,35 +260,30 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
     const uint32_t kv0 = ptx::smem_u32(smem + C::kKvOff);
     const uint32_t q0 = ptx::smem_u32(smem + C::kQOff);
     const uint32_t p0 = ptx::smem_u32(smem + C::kPOff);
-    constexpr uint32_t idesc_qk = kFp8 ? ptx::instr_desc(0, 0, 0, 0, kTileM, kN)
-                                       : ptx::instr_desc(1, 1, 0, 0, kTileM, kN);
-    constexpr uint32_t idesc_pv = kFp8 ? ptx::instr_desc(0, 0, 1, 1, kTileM, kN)
-                                       : ptx::instr_desc(1, 1, 1, 1, kTileM, kN);
+    constexpr uint32_t idesc_qk = kFp8 ? ptx::instr_desc(0, 0, 0, 0, kTileM, C::kNMma)
+                                       : ptx::instr_desc(1, 1, 0, 0, kTileM, C::kNMma);
+    constexpr uint32_t idesc_pv = kFp8 ? ptx::instr_desc(0, 0, 1, 1, kTileM, C::kNMma)
+                                       : ptx::instr_desc(1, 1, 1, 1, kTileM, C::kNMma);
     uint32_t g = 0, pi = 0;
 
     auto issue_qk = [&](uint32_t gg) {
         const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
-        const uint32_t d = tmem + ((gg & 1) ? kColS1 : kColS0);
+        const uint32_t d = tmem + ((gg % C::kSBufs) ? C::kColS1 : 0u);
         if constexpr (kFp8) {
-            uint32_t acc = 0;
+            // N = 96: query rows 0-47 hold hi, 48-95 hold lo
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t qb = q0 + part * C::kQPart;
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        uint64_t a = ptx::smem_desc(st + c * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                        uint64_t b = ptx::smem_desc(qb + c * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                        ptx::mma_f8(d, a, b, idesc_qk, acc);
-                        acc = 1;
-                    }
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    uint64_t a = ptx::smem_desc(st + 4 * C::kChunkBytes + ks * 32, 16, 512, ptx::kSwizzle64B);
-                    uint64_t b = ptx::smem_desc(qb + 4 * C::kQChunk + ks * 32, 16, 512, ptx::kSwizzle64B);
-                    ptx::mma_f8(d, a, b, idesc_qk, 1);
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint64_t a = ptx::smem_desc(st + c * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    uint64_t b = ptx::smem_desc(q0 + c * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    ptx::mma_f8(d, a, b, idesc_qk, (c | ks) ? 1u : 0u);
                 }
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                uint64_t a = ptx::smem_desc(st + 4 * C::kChunkBytes + ks * 32, 16, 512, ptx::kSwizzle64B);
+                uint64_t b = ptx::smem_desc(q0 + C::kQRopeOff + ks * 32, 16, 512, ptx::kSwizzle64B);
+                ptx::mma_f8(d, a, b, idesc_qk, 1u);
             }
         } else {
 #pragma unroll
@@ -278,15 +301,13 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
         const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            const uint32_t d = tmem + kColO + 64 * m;
+            const uint32_t d = tmem + C::kColO + C::kOStride * m;
             if constexpr (kFp8) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {  // 32 positions per MMA; P = hi + lo
+                for (int ks = 0; ks < 4; ++ks) {  // 32 positions per MMA; N = 96: P hi | P lo
                     uint64_t a = ptx::smem_desc(st + m * C::kChunkBytes + ks * 4096, 16384, 1024, ptx::kSwizzle128B);
-                    uint64_t bh = ptx::smem_desc(p0 + ks * 512, 128, 2048, ptx::kSwizzleNone);
-                    uint64_t bl = ptx::smem_desc(p0 + C::kPPart + ks * 512, 128, 2048, ptx::kSwizzleNone);
-                    ptx::mma_f8(d, a, bh, idesc_pv, (first && ks == 0) ? 0u : 1u);
-                    ptx::mma_f8(d, a, bl, idesc_pv, 1u);
+                    uint64_t b = ptx::smem_desc(p0 + ks * 512, 128, 2048, ptx::kSwizzleNone);
+                    ptx::mma_f8(d, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
                 }
             } else {
 #pragma unroll
@@ -303,44 +324,51 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
         if (nt == 0 || aborted(ms)) return;
-        if (!waitb(p, ms, &ms.q_ready, pi & 1)) return;
-        ptx::tc_fence_after();
         const uint32_t g0 = g;
-        auto do_qk = [&](int k) -> bool {
-            const uint32_t gg = g0 + k;
-            if (!waitb(p, ms, &ms.kv_full[gg % C::kStages], (gg / C::kStages) & 1)) return false;
-            if (!waitb(p, ms, &ms.s_free[gg & 1], ((gg >> 1) & 1) ^ 1)) return false;
-            ptx::tc_fence_after();
-            if (lane == 0) {
-                issue_qk(gg);
-                ptx::mma_commit(&ms.s_full[gg & 1]);
+        int nq = 0, npv = 0;           // tiles whose scores / values have been issued
+        bool q_ok = false, o_ok = false;
+        uint64_t t_idle = ptx::globaltimer();
+        // Issue each MMA group as soon as its operands are ready: the values of
+        // tile k as soon as its weights are written (so its KV stage frees at
+        // once), the scores of tile k as soon as it has landed.
+        while (npv < nt) {
+            bool progress = false;
+            if (npv < nq) {
+                const uint32_t gp = g0 + npv;
+                if (!o_ok && npv == 0) o_ok = ptx::mbar_test(&ms.o_free, (pi & 1) ^ 1);
+                if ((npv > 0 || o_ok) && ptx::mbar_test(&ms.p_full, gp & 1)) {
+                    ptx::tc_fence_after();
+                    if (lane == 0) {
+                        issue_pv(gp, npv == 0);
+                        ptx::mma_commit(&ms.kv_empty[gp % C::kStages]);
+                        ptx::mma_commit(&ms.pv_done);
+                    }
+                    __syncwarp();
+                    ++npv;
+                    progress = true;
+                }
             }
-            __syncwarp();
-            return true;
-        };
-        auto do_pv = [&](int k) -> bool {
-            const uint32_t gp = g0 + k;
-            if (!waitb(p, ms, &ms.p_full, gp & 1)) return false;
-            if (k == 0 && !waitb(p, ms, &ms.o_free, (pi & 1) ^ 1)) return false;
-            ptx::tc_fence_after();
-            if (lane == 0) {
-                issue_pv(gp, k == 0);
-                ptx::mma_commit(&ms.kv_empty[gp % C::kStages]);
-                ptx::mma_commit(&ms.pv_done);
+            if (nq < nt) {
+                const uint32_t gq = g0 + nq;
+                if (!q_ok) q_ok = ptx::mbar_test(&ms.q_ready, pi & 1);
+                if (q_ok && ptx::mbar_test(&ms.kv_full[gq % C::kStages], (gq / C::kStages) & 1) &&
+                    ptx::mbar_test(&ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1)) {
+                    ptx::tc_fence_after();
+                    if (lane == 0) {
+                        issue_qk(gq);
+                        ptx::mma_commit(&ms.s_full[gq % C::kSBufs]);
+                    }
+                    __syncwarp();
+                    ++nq;
+                    progress = true;
+                }
             }
-            __syncwarp();
-            return true;
-        };
-        // With two KV stages the scores of tile k are issued before the values
-        // of tile k-1, so the tensor core works while the softmax runs; with
-        // one stage, tile k can only land after tile k-1's values are done.
-        for (int k = 0; k <= nt; ++k) {
-            if (C::kStages > 1) {
-                if (k < nt && !do_qk(k)) return;
-                if (k > 0 && !do_pv(k - 1)) return;
-            } else {
-                if (k > 0 && !do_pv(k - 1)) return;
-                if (k < nt && !do_qk(k)) return;
+            const uint64_t now = ptx::globaltimer();
+            if (progress) {
+                t_idle = now;
+            } else if (now - t_idle > kWaitLimitNs || aborted(ms)) {
+                cta_abort(p, ms);
+                return;
             }
         }
         g = g0 + nt;
@@ -353,7 +381,7 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
 }
 
 // ---------------------------------------------------------------------------
-// warps 2-5: query staging, online softmax, epilogue
+// warps 2-9: query staging, online softmax, epilogue
 // ---------------------------------------------------------------------------
 template <bool kFp8>
 __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int b, int r0, int st,
@@ -393,7 +421,7 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
         const float qscale = ldexpf(1.f, e2);
         const float inv = ldexpf(1.f, -e2);
         if (st == 0) ms.qscale = qscale;
-        // pass 2: hi = e4m3(q/s), lo = e4m3(q/s - hi), in the MMA's K-major layouts
+        // pass 2: hi rows 0-47 and lo rows 48-95 of the K-major operand
         for (int u = st; u < kN * 36; u += kSoftmaxThreads) {
             const int row = u / 36, uu = u % 36;
             uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
@@ -415,16 +443,16 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
                     }
                 }
             }
-            int off;
+            const int rl = row + kN;   // lo row
             if (uu < 32) {
                 const int c = uu >> 3, k = uu & 7;
-                off = c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4)) = hi4;
+                *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + rl * 128 + ((k ^ (rl & 7)) << 4)) = lo4;
             } else {
                 const int k = uu - 32;
-                off = 4 * C::kQChunk + row * 64 + ((k ^ ((row >> 1) & 3)) << 4);
+                *reinterpret_cast<uint4 *>(qs + C::kQRopeOff + row * 64 + ((k ^ ((row >> 1) & 3)) << 4)) = hi4;
+                *reinterpret_cast<uint4 *>(qs + C::kQRopeOff + rl * 64 + ((k ^ ((rl >> 1) & 3)) << 4)) = lo4;
             }
-            *reinterpret_cast<uint4 *>(qs + off) = hi4;
-            *reinterpret_cast<uint4 *>(qs + C::kQPart + off) = lo4;
         }
     } else {
         for (int u = st; u < kN * 72; u += kSoftmaxThreads) {
@@ -442,12 +470,25 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
     return true;
 }
 
+// 24 rows of one accumulator column block; for FP8 the hi and lo halves
+// (48 columns apart) are added.
+template <bool kFp8>
+__device__ __forceinline__ void tmem_rows24(uint32_t taddr, float *v) {
+    ptx::tmem_ld24(taddr, v);
+    if constexpr (kFp8) {
+        float w[kHalf];
+        ptx::tmem_ld24(taddr + kN, w);
+#pragma unroll
+        for (int c = 0; c < kHalf; ++c) v[c] += w[c];
+    }
+}
+
 template <bool kFp8>
 __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, int slot, int g_idx) {
     using C = Cfg<kFp8>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int w8 = warp - 2;                   // 0..7
-    const int h = w8 >> 2;                     // column half: columns [24h, 24h + 24)
+    const int h = w8 >> 2;                     // row half: rows [24h, 24h + 24)
     const int w4 = w8 & 3;                     // warp within the half
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int i = quad * 32 + lane;            // tile position / TMEM lane
@@ -456,14 +497,14 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
     const int cb = h * kHalf;
     const uint32_t tmem = ms.tmem_base + ((uint32_t)(quad * 32) << 16);
     const int r0 = g_idx * kN;
-    constexpr float kEmpty = -1e30f;           // stabiliser of a column that has seen nothing yet
+    constexpr float kEmpty = -1e30f;           // stabiliser of a row that has seen nothing yet
     uint32_t g = 0;
     GroupSync all_sync(&ms.all_sync), hsync(&ms.half_sync[h]);
 
     for_each_piece(p, slot, [&](const Piece &pc) {
         if (aborted(ms)) return;
         const int nt = ntiles_of(pc);
-        // visible positions per column, limited to this piece's pages
+        // visible positions per row, limited to this piece's pages
         if (st < kN) {
             const int r = r0 + st;
             int lim = 0, bad = 0;
@@ -484,7 +525,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (st == 0 && pc.bad_ctx && g_idx == 0) report_error(p.err, MLA_DEV_BAD_CTX, pc.b);
         if (!all_sync(p, ms)) return;
         const int rows_here = min(kN, p.R - r0);
-        int min_lim = INT_MAX;  // over this half's real columns
+        int min_lim = INT_MAX;  // over this half's real rows
         for (int c = cb; c < min(cb + kHalf, rows_here); ++c) min_lim = min(min_lim, ms.col_lim[c]);
 
         if (nt == 0) {  // nothing to read: write the empty (or invalid) result
@@ -520,13 +561,14 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             if (!waitb(p, ms, &ms.kv_full[stage], (gg / C::kStages) & 1)) return;
             const uint32_t info = ms.stage_info[stage];
             piece_bad |= (info >> 31) != 0;
-            if (!waitb(p, ms, &ms.s_full[gg & 1], (gg >> 1) & 1)) return;
+            const int sb = gg % C::kSBufs;
+            if (!waitb(p, ms, &ms.s_full[sb], (gg / C::kSBufs) & 1)) return;
             ptx::tc_fence_after();
             float s[kHalf];
-            ptx::tmem_ld24(tmem + ((gg & 1) ? kColS1 : kColS0) + cb, s);
+            tmem_rows24<kFp8>(tmem + (sb ? C::kColS1 : 0u) + cb, s);
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&ms.s_free[gg & 1]);
+            if (lane == 0) ptx::mbar_arrive(&ms.s_free[sb]);
 
             const int pos0 = (pc.page_lo + k * kTilePages) * kPage;
             const int pos = pos0 + i;
@@ -576,17 +618,20 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 }
                 if (!hsync(p, ms)) return;  // red[] reads done before any reuse
                 if (moved && k > 0) {
-                    // O^T holds earlier tiles: wait for their value MMA, then rescale columns
+                    // O^T holds earlier tiles: wait for their value MMA, then rescale rows
                     if (!waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
                     ptx::tc_fence_after();
 #pragma unroll 1
                     for (int m = 0; m < 4; ++m) {
-                        float o[kHalf];
-                        const uint32_t oc = tmem + kColO + 64 * m + cb;
-                        ptx::tmem_ld24(oc, o);
+#pragma unroll 1
+                        for (int part = 0; part < (kFp8 ? 2 : 1); ++part) {
+                            float o[kHalf];
+                            const uint32_t oc = tmem + C::kColO + C::kOStride * m + part * kN + cb;
+                            ptx::tmem_ld24(oc, o);
 #pragma unroll
-                        for (int c = 0; c < kHalf; ++c) o[c] *= alpha[c];
-                        ptx::tmem_st24(oc, o);
+                            for (int c = 0; c < kHalf; ++c) o[c] *= alpha[c];
+                            ptx::tmem_st24(oc, o);
+                        }
                     }
                 }
             }
@@ -630,17 +675,18 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     lw[w] = lp[0] | (lp[1] << 16);
                 }
                 // 16-row groups: half 0 owns group 0 and the low 8 bytes of group 1,
-                // half 1 the high 8 bytes of group 1 and group 2
-                unsigned char *g16 = pb + (h == 0 ? 0 : 4096) + i * 16;
-                unsigned char *g8 = pb + 2048 + i * 16 + (h == 0 ? 0 : 8);
-                const int w16 = h == 0 ? 0 : 2, w8o = h == 0 ? 4 : 0;
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t *src = part ? lw : hw;
-                    const int off = part ? C::kPPart : 0;
-                    *reinterpret_cast<uint4 *>(g16 + off) =
-                        make_uint4(src[w16], src[w16 + 1], src[w16 + 2], src[w16 + 3]);
-                    *reinterpret_cast<uint2 *>(g8 + off) = make_uint2(src[w8o], src[w8o + 1]);
+                // half 1 the high 8 bytes of group 1 and group 2 (lo: groups 3-5)
+                if (h == 0) {
+                    *reinterpret_cast<uint4 *>(pb + i * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint2 *>(pb + 2048 + i * 16) = make_uint2(hw[4], hw[5]);
+                    *reinterpret_cast<uint4 *>(pb + C::kPLoOff + i * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    *reinterpret_cast<uint2 *>(pb + C::kPLoOff + 2048 + i * 16) = make_uint2(lw[4], lw[5]);
+                } else {
+                    *reinterpret_cast<uint2 *>(pb + 2048 + i * 16 + 8) = make_uint2(hw[0], hw[1]);
+                    *reinterpret_cast<uint4 *>(pb + 4096 + i * 16) = make_uint4(hw[2], hw[3], hw[4], hw[5]);
+                    *reinterpret_cast<uint2 *>(pb + C::kPLoOff + 2048 + i * 16 + 8) = make_uint2(lw[0], lw[1]);
+                    *reinterpret_cast<uint4 *>(pb + C::kPLoOff + 4096 + i * 16) =
+                        make_uint4(lw[2], lw[3], lw[4], lw[5]);
                 }
             } else {
 #pragma unroll
@@ -688,7 +734,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
             float o[kHalf];
-            ptx::tmem_ld24(tmem + kColO + 64 * m + cb, o);
+            tmem_rows24<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
             const int d = 128 * m + i;
             for (int c = 0; c < ncols; ++c) {
                 const float v = o[c] * ms.inv_l[cb + c];
@@ -831,10 +877,10 @@ int launch_impl(const Problem &p, cudaStream_t stream) {
 
 static_assert(smem_bytes<true>() <= 232448, "FP8 tile does not fit shared memory");
 static_assert(smem_bytes<false>() <= 232448, "bf16 tile does not fit shared memory");
+static_assert(Cfg<true>::kColO + 3 * Cfg<true>::kOStride + Cfg<true>::kNMma <= kTmemCols, "TMEM overflow");
+static_assert(Cfg<false>::kColO + 3 * Cfg<false>::kOStride + Cfg<false>::kNMma <= kTmemCols, "TMEM overflow");
 
 }  // namespace
-
-int tc_rows_per_group() { return kN; }
 
 int launch_tc(const Problem &p, cudaStream_t stream) {
     if (p.rows_per_group != kN) return MLA_ERR_INVALID_ARG;
