@@ -151,6 +151,33 @@ MLA_API int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages
                mla_stream_t stream);
 
 /*
+ * mla_decode without a caller-provided workspace, for callers that cannot
+ * allocate device memory when they decode (for example while a CUDA graph is
+ * captured in a mode that forbids allocation, or inside a runtime whose device
+ * memory all belongs to another allocator).  The pages describe no such
+ * entry point; it is a service of this library, not part of the method.
+ *
+ * Same arguments and results as mla_decode, minus the workspace.  The scratch
+ * is one fixed 32 MiB array in device memory, defined in the library, held by
+ * every GPU that loads the library until the process exits.  The call
+ * allocates and frees nothing:
+ *   - If mla_decode_workspace_size(dims) exceeds 32 MiB it returns
+ *     MLA_ERR_WORKSPACE and launches nothing.
+ *   - The first call on each device looks up the array's device address (a
+ *     host-side runtime query, made with that device current).  Make that
+ *     first call before any stream capture on the device.
+ *   - Each call clears the array's error word on `stream`, then runs the
+ *     decode there.  The device error word is not reported.
+ *   - All calls share the one array, so calls that can overlap on the GPU
+ *     (different streams, or several host threads) race and corrupt each
+ *     other's results.  Serialise them, e.g. on one stream.
+ */
+MLA_API int mla_decode_noalloc(const void *q_lat, const void *q_pe, const void *kv_pages,
+                               const float *kv_scale, const int32_t *page_table,
+                               const int32_t *ctx_lens, float sm_scale, void *out, float *lse,
+                               const mla_dims *dims, mla_stream_t stream);
+
+/*
  * Exact merge of partial attention results over disjoint position sets
  * (split-KV pieces, or context-parallel ranks each holding a subset of the
  * positions): "Inside Kimi K3 optimisation work", section 1, DCP -- each

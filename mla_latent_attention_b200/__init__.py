@@ -29,7 +29,7 @@ KV_BF16, KV_FP8 = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 KERNELS = {"auto": 0, "simt": 1, "tcgen05": 2}
 DEV_ERRORS = {0: "ok", 1: "bad page index", 2: "bad context length", 3: "bad visible count"}
-EXPORTED = ("mla_decode_workspace_size", "mla_decode", "mla_merge_partials",
+EXPORTED = ("mla_decode_workspace_size", "mla_decode", "mla_decode_noalloc", "mla_merge_partials",
             "mla_read_device_error", "mla_reset_device_error", "mla_status_string",
             "mla_last_cuda_error")
 
@@ -68,6 +68,9 @@ def load_library(path: str = None):
         lib.mla_decode.restype = ctypes.c_int
         lib.mla_decode.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                    ctypes.POINTER(Dims), vp, ctypes.c_size_t, vp]
+        lib.mla_decode_noalloc.restype = ctypes.c_int
+        lib.mla_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                           ctypes.POINTER(Dims), vp]
         lib.mla_merge_partials.restype = ctypes.c_int
         lib.mla_merge_partials.argtypes = [vp, vp, i32, i64, vp, i32, vp, vp]
         lib.mla_read_device_error.restype = ctypes.c_int

@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation, workspace layout, kernel dispatch.
 #include <atomic>
 #include <cstring>
+#include <mutex>
 
 #include "mla_common.cuh"
 
@@ -160,6 +161,70 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     }
     if (pl.n_slots > 1) rc = launch_merge_internal(p, s);
     return rc;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.
+//
+// Some callers cannot call cudaMalloc (or any allocating routine) at the point
+// where they decode: code running while a CUDA graph is being captured in a
+// mode that forbids allocation, runtimes whose device memory is entirely
+// owned by another allocator arena, or plugins that must not grow the
+// process's device footprint per call.  For them the library keeps one fixed
+// scratch array in device memory (every GPU that loads the library holds it
+// until the process exits) and runs the ordinary decode with that array as
+// its workspace.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static constexpr int kMaxDevices = 64;
+static void *g_noalloc_ptr[kMaxDevices];
+static std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  The host-side
+// symbol is only a stand-in: the address must come from the runtime, once per
+// device, with that device current.
+static int noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return MLA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || !ptr) {
+            note_cuda_error(e);
+            return MLA_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MLA_OK;
+}
+
+int mla_decode_noalloc(const void *q_lat, const void *q_pe, const void *kv_pages, const float *kv_scale,
+                       const int32_t *page_table, const int32_t *ctx_lens, float sm_scale, void *out,
+                       float *lse, const mla_dims *dims, mla_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    const int64_t need = mla_decode_workspace_size(dims);
+    if (need < 0) return (int)need;
+    if ((size_t)need > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE;
+    void *ws = nullptr;
+    rc = noalloc_scratch(&ws);
+    if (rc) return rc;
+    // the array keeps the previous call's contents: the error word must start clear
+    cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeaderBytes, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return MLA_ERR_CUDA;
+    }
+    return mla_decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, out, lse, dims, ws,
+                      kNoAllocScratchBytes, stream);
 }
 
 int mla_merge_partials(const float *out_parts, const float *lse_parts, int32_t n_parts, int64_t rows,
