@@ -91,20 +91,28 @@ struct Cfg {
     static constexpr int kPBytes = (kNMma / kPGroupRows) * kTileM * 16;           // 12288 both
     static constexpr int kPLoOff = kFp8 ? (kN / 16) * kTileM * 16 : 0;             // lo rows start (group 3)
     static constexpr int kMiscOff = kPOff + kPBytes;
-    static constexpr int kPageBytes = kFp8 ? (4 * 2048 + 1024 + 64) : 9 * 2048;   // bytes a page brings
+    // Each stage is filled and freed in parts: the value chunks (FP8 4 x 128
+    // dims, bf16 8 x 64 dims) and the RoPE chunk, so the next tile's copies
+    // start as soon as the previous tile's MMAs are done with each part.
+    static constexpr int kParts = kVChunks + 1;
+    static constexpr int kRope = kVChunks;                                        // part index of the RoPE chunk
+    __host__ __device__ static constexpr uint32_t part_bytes(int part) {            // per page
+        return kFp8 ? (part == kRope ? 1024u : (part == 0 ? 2048u + 64u : 2048u)) : 2048u;
+    }
     // exponent offset C and lazy threshold TAU of the softmax stabiliser
     static constexpr float kC = kFp8 ? 4.5f : 0.f;
     static constexpr float kTau = kFp8 ? 4.f : 8.f;
 };
 
 struct Misc {
-    uint64_t kv_full[2], kv_empty[2], s_full[2], s_free[2];
+    uint64_t part_full[2][9], part_empty[2][9];   // per KV stage and part
+    uint64_t s_full[2], s_free[2];
     uint64_t p_full, pv_done, q_ready, o_free, drain;
     uint64_t all_sync;        // the eight softmax warps (bounded waits, unlike bar.sync)
     uint64_t half_sync[2];    // the four softmax warps of each row half
     uint32_t tmem_base;
     int abort;
-    uint32_t stage_info[2];   // bit i: page slot i loaded; bit 31: a page of the tile was invalid
+    uint32_t stage_info[4];   // per tile mod 4: bit i page slot i loaded; bit 31 a page was invalid
     int vote[2][2][4];        // [half][tile parity][warp]
     int col_lim[kN];          // positions visible to row r within this piece, 0 = none
     int col_bad[kN];
@@ -206,7 +214,7 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
         for (int k = 0; k < nt; ++k, ++g) {
             if (aborted(ms)) return;
             const int stage = g % C::kStages;
-            if (!waitb(p, ms, &ms.kv_empty[stage], ((g / C::kStages) & 1) ^ 1)) return;
+            const uint32_t empty_parity = ((g / C::kStages) & 1) ^ 1;
             const int pg0 = pc.page_lo + k * kTilePages;
             const int npg = min(kTilePages, pc.page_hi - pg0);
             int pid = -1;
@@ -219,26 +227,30 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
             const unsigned badm = __ballot_sync(0xffffffffu, lane < npg && !ok);
             if (lane == 0) {
                 if (badm) report_error(p.err, MLA_DEV_BAD_PAGE, pc.b);
-                ms.stage_info[stage] = okm | (badm ? 0x80000000u : 0u);
-                ptx::mbar_arrive_expect_tx(&ms.kv_full[stage], __popc(okm) * C::kPageBytes);
+                ms.stage_info[g & 3] = okm | (badm ? 0x80000000u : 0u);
             }
-            __syncwarp();
-            if (ok) {
-                unsigned char *st = smem + C::kKvOff + stage * C::kStageBytes;
-                const int y = pid * kPage;
+            const uint32_t n_ok = __popc(okm);
+            unsigned char *st = smem + C::kKvOff + stage * C::kStageBytes;
+            const int y = pid * kPage;
+            // RoPE first (freed first, right after the previous scores), then the value chunks
+            for (int q = 0; q < C::kParts; ++q) {
+                const int part = q == 0 ? C::kRope : q - 1;
+                if (!waitb(p, ms, &ms.part_empty[stage][part], empty_parity)) return;
+                if (lane == 0) ptx::mbar_arrive_expect_tx(&ms.part_full[stage][part], n_ok * C::part_bytes(part));
+                __syncwarp();
+                if (!ok) continue;
+                uint64_t *bar = &ms.part_full[stage][part];
                 if constexpr (kFp8) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        ptx::tma_load_2d(st + c * C::kChunkBytes + lane * 2048, map_a, &ms.kv_full[stage],
-                                         128 * c, y);
-                    ptx::tma_load_2d(st + 4 * C::kChunkBytes + lane * 1024, map_b, &ms.kv_full[stage], 512, y);
-                    ptx::bulk_load(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
-                                   p.kv_scale + (int64_t)pid * kPage, 64, &ms.kv_full[stage]);
+                    if (part == C::kRope) {
+                        ptx::tma_load_2d(st + 4 * C::kChunkBytes + lane * 1024, map_b, bar, 512, y);
+                    } else {
+                        ptx::tma_load_2d(st + part * C::kChunkBytes + lane * 2048, map_a, bar, 128 * part, y);
+                        if (part == 0)
+                            ptx::bulk_load(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
+                                           p.kv_scale + (int64_t)pid * kPage, 64, bar);
+                    }
                 } else {
-#pragma unroll
-                    for (int c = 0; c < 9; ++c)
-                        ptx::tma_load_2d(st + c * C::kChunkBytes + lane * 2048, map_a, &ms.kv_full[stage],
-                                         64 * c, y);
+                    ptx::tma_load_2d(st + part * C::kChunkBytes + lane * 2048, map_a, bar, 64 * part, y);
                 }
             }
             if (k + kPrefetchAhead < nt) prefetch_tile(pc, k + kPrefetchAhead);
@@ -246,7 +258,8 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
     });
     // make sure no copy is still landing when the CTA leaves
     for (uint32_t h = g > (uint32_t)C::kStages ? g - C::kStages : 0; h < g; ++h)
-        ptx::mbar_wait(&ms.kv_full[h % C::kStages], (h / C::kStages) & 1, kWaitLimitNs);
+        for (int part = 0; part < C::kParts; ++part)
+            ptx::mbar_wait(&ms.part_full[h % C::kStages][part], (h / C::kStages) & 1, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------
@@ -266,39 +279,41 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                                        : ptx::instr_desc(1, 1, 1, 1, kTileM, C::kNMma);
     uint32_t g = 0, pi = 0;
 
-    auto issue_qk = [&](uint32_t gg) {
+    // Score MMAs reading one part of the tile (accumulate from the second MMA of the tile on).
+    auto issue_qk_part = [&](uint32_t gg, int part, bool first) {
         const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
         const uint32_t d = tmem + ((gg % C::kSBufs) ? C::kColS1 : 0u);
         if constexpr (kFp8) {
             // N = 96: query rows 0-47 hold hi, 48-95 hold lo
+            if (part == C::kRope) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint64_t a = ptx::smem_desc(st + 4 * C::kChunkBytes + ks * 32, 16, 512, ptx::kSwizzle64B);
+                    uint64_t b = ptx::smem_desc(q0 + C::kQRopeOff + ks * 32, 16, 512, ptx::kSwizzle64B);
+                    ptx::mma_f8(d, a, b, idesc_qk, (first && ks == 0) ? 0u : 1u);
+                }
+            } else {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    uint64_t a = ptx::smem_desc(st + c * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                    uint64_t b = ptx::smem_desc(q0 + c * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                    ptx::mma_f8(d, a, b, idesc_qk, (c | ks) ? 1u : 0u);
+                    uint64_t a = ptx::smem_desc(st + part * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    uint64_t b = ptx::smem_desc(q0 + part * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    ptx::mma_f8(d, a, b, idesc_qk, (first && ks == 0) ? 0u : 1u);
                 }
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                uint64_t a = ptx::smem_desc(st + 4 * C::kChunkBytes + ks * 32, 16, 512, ptx::kSwizzle64B);
-                uint64_t b = ptx::smem_desc(q0 + C::kQRopeOff + ks * 32, 16, 512, ptx::kSwizzle64B);
-                ptx::mma_f8(d, a, b, idesc_qk, 1u);
             }
         } else {
 #pragma unroll
-            for (int c = 0; c < 9; ++c)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    uint64_t a = ptx::smem_desc(st + c * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                    uint64_t b = ptx::smem_desc(q0 + c * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                    ptx::mma_f16(d, a, b, idesc_qk, (c | ks) ? 1u : 0u);
-                }
+            for (int ks = 0; ks < 4; ++ks) {
+                uint64_t a = ptx::smem_desc(st + part * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                uint64_t b = ptx::smem_desc(q0 + part * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                ptx::mma_f16(d, a, b, idesc_qk, (first && ks == 0) ? 0u : 1u);
+            }
         }
     };
 
+    // Value MMAs; each 128-dim block frees its value chunk(s) of the stage as it completes.
     auto issue_pv = [&](uint32_t gg, bool first) {
-        const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
+        const int stage = gg % C::kStages;
+        const uint32_t st = kv0 + stage * C::kStageBytes;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const uint32_t d = tmem + C::kColO + C::kOStride * m;
@@ -318,29 +333,42 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                     ptx::mma_f16(d, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
                 }
             }
+            if constexpr (kFp8) {
+                ptx::mma_commit(&ms.part_empty[stage][m]);
+            } else {
+                ptx::mma_commit(&ms.part_empty[stage][2 * m]);
+                ptx::mma_commit(&ms.part_empty[stage][2 * m + 1]);
+            }
         }
+    };
+
+    // Barrier tests are made by lane 0 and broadcast, so the warp never diverges
+    // on a phase that completes while it polls.
+    auto test = [&](uint64_t *bar, uint32_t parity) -> bool {
+        const int r = lane == 0 ? (int)ptx::mbar_test(bar, parity) : 0;
+        return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
 
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
         if (nt == 0 || aborted(ms)) return;
         const uint32_t g0 = g;
-        int nq = 0, npv = 0;           // tiles whose scores / values have been issued
-        bool q_ok = false, o_ok = false;
+        int nq = 0, qp = 0, npv = 0;   // tiles whose scores / values are issued; parts of tile nq issued
+        bool q_ok = false, o_ok = false, s_ok = false;
         uint64_t t_idle = ptx::globaltimer();
         // Issue each MMA group as soon as its operands are ready: the values of
-        // tile k as soon as its weights are written (so its KV stage frees at
-        // once), the scores of tile k as soon as it has landed.
+        // tile k as soon as its weights are written (each value block then
+        // frees its chunk for the next copy), the scores of tile k part by part
+        // as the parts land.
         while (npv < nt) {
             bool progress = false;
             if (npv < nq) {
                 const uint32_t gp = g0 + npv;
-                if (!o_ok && npv == 0) o_ok = ptx::mbar_test(&ms.o_free, (pi & 1) ^ 1);
-                if ((npv > 0 || o_ok) && ptx::mbar_test(&ms.p_full, gp & 1)) {
+                if (!o_ok && npv == 0) o_ok = test(&ms.o_free, (pi & 1) ^ 1);
+                if ((npv > 0 || o_ok) && test(&ms.p_full, gp & 1)) {
                     ptx::tc_fence_after();
                     if (lane == 0) {
                         issue_pv(gp, npv == 0);
-                        ptx::mma_commit(&ms.kv_empty[gp % C::kStages]);
                         ptx::mma_commit(&ms.pv_done);
                     }
                     __syncwarp();
@@ -350,25 +378,38 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
             }
             if (nq < nt) {
                 const uint32_t gq = g0 + nq;
-                if (!q_ok) q_ok = ptx::mbar_test(&ms.q_ready, pi & 1);
-                if (q_ok && ptx::mbar_test(&ms.kv_full[gq % C::kStages], (gq / C::kStages) & 1) &&
-                    ptx::mbar_test(&ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1)) {
+                const int stage = gq % C::kStages;
+                if (!q_ok) q_ok = test(&ms.q_ready, pi & 1);
+                if (q_ok && qp == 0 && !s_ok) s_ok = test(&ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1);
+                while (q_ok && s_ok && qp < C::kParts) {
+                    const int part = qp == 0 ? C::kRope : qp - 1;
+                    if (!test(&ms.part_full[stage][part], (gq / C::kStages) & 1)) break;
                     ptx::tc_fence_after();
+                    if (lane == 0) issue_qk_part(gq, part, qp == 0);
+                    __syncwarp();
+                    ++qp;
+                    progress = true;
+                }
+                if (qp == C::kParts) {
                     if (lane == 0) {
-                        issue_qk(gq);
                         ptx::mma_commit(&ms.s_full[gq % C::kSBufs]);
+                        ptx::mma_commit(&ms.part_empty[stage][C::kRope]);  // RoPE is read by scores only
                     }
                     __syncwarp();
                     ++nq;
-                    progress = true;
+                    qp = 0;
+                    s_ok = false;
                 }
             }
-            const uint64_t now = ptx::globaltimer();
             if (progress) {
-                t_idle = now;
-            } else if (now - t_idle > kWaitLimitNs || aborted(ms)) {
-                cta_abort(p, ms);
-                return;
+                if (lane == 0) t_idle = ptx::globaltimer();
+            } else {
+                int expired = 0;
+                if (lane == 0) expired = (ptx::globaltimer() - t_idle > kWaitLimitNs) || aborted(ms);
+                if (__shfl_sync(0xffffffffu, expired, 0)) {
+                    cta_abort(p, ms);
+                    return;
+                }
             }
         }
         g = g0 + nt;
@@ -383,6 +424,12 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
 // ---------------------------------------------------------------------------
 // warps 2-9: query staging, online softmax, epilogue
 // ---------------------------------------------------------------------------
+// Stages the 48 query rows of this group as the score MMA's B operand
+// (K-major, 128B / 64B swizzled chunks).  FP8: one pass into registers, the
+// block's largest |q| sets a power-of-two scale s, then hi = e4m3(q/s) goes to
+// rows 0-47 and lo = e4m3(q/s - hi) to rows 48-95.  A power-of-two s keeps q/s
+// a bf16 value, which hi + lo represents exactly (short of e4m3 underflow far
+// below the largest q).  Rows past R are zero.
 template <bool kFp8>
 __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int b, int r0, int st,
                            GroupSync &gsync) {
@@ -390,21 +437,28 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
     const int64_t qrow0 = (int64_t)b * p.R;
     unsigned char *qs = smem + C::kQOff;
     if constexpr (kFp8) {
-        // pass 1: the block's largest |q| sets the e4m3 scale
+        // unit = 16 consecutive dims of one row (36 units per row, 32 latent + 4 RoPE)
+        constexpr int kUnits = kN * 36;
+        constexpr int kPer = (kUnits + kSoftmaxThreads - 1) / kSoftmaxThreads;  // 7
+        uint4 v[kPer][2];
         float amax = 0.f;
-        for (int u = st; u < kN * 36; u += kSoftmaxThreads) {
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int u = st + j * kSoftmaxThreads;
             const int row = u / 36, uu = u % 36;
-            if (r0 + row >= p.R) continue;
-            const __nv_bfloat16 *src = uu < 32 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 16
-                                               : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 32) * 16;
-            const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+            v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
+            if (u < kUnits && r0 + row < p.R) {
+                const __nv_bfloat16 *src = uu < 32 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 16
+                                                   : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 32) * 16;
+                v[j][0] = __ldg(reinterpret_cast<const uint4 *>(src));
+                v[j][1] = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint4 v = __ldg(s4 + h);
-                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v[j][h]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float2 f = __bfloat1622float2(b2[e]);
+                    const float2 f = __bfloat1622float2(b2[e]);
                     amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
                 }
             }
@@ -414,35 +468,33 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
         if (!gsync(p, ms)) return false;
 #pragma unroll
         for (int w = 0; w < 8; ++w) amax = fmaxf(amax, ms.amax[w]);
-        // A power-of-two scale keeps q/s a bf16 value, which hi + lo then
-        // represents exactly (short of e4m3 underflow far below the largest q).
         int e2 = 0;
         if (amax > 0.f) frexpf(amax / 448.f, &e2);
-        const float qscale = ldexpf(1.f, e2);
         const float inv = ldexpf(1.f, -e2);
-        if (st == 0) ms.qscale = qscale;
-        // pass 2: hi rows 0-47 and lo rows 48-95 of the K-major operand
-        for (int u = st; u < kN * 36; u += kSoftmaxThreads) {
+        if (st == 0) ms.qscale = ldexpf(1.f, e2);
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int u = st + j * kSoftmaxThreads;
+            if (u >= kUnits) continue;
             const int row = u / 36, uu = u % 36;
-            uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
-            if (r0 + row < p.R) {
-                const __nv_bfloat16 *src = uu < 32 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 16
-                                                   : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 32) * 16;
-                const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-                uint8_t *hv = reinterpret_cast<uint8_t *>(&hi4);
-                uint8_t *lv = reinterpret_cast<uint8_t *>(&lo4);
+            uint32_t hw[4], lw[4];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint4 v = __ldg(s4 + h);
-                    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+            for (int h = 0; h < 2; ++h) {
+                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v[j][h]);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(b2[e]);
-                        split_e4m3(f.x * inv, hv[8 * h + 2 * e], lv[8 * h + 2 * e]);
-                        split_e4m3(f.y * inv, hv[8 * h + 2 * e + 1], lv[8 * h + 2 * e + 1]);
-                    }
+                for (int q = 0; q < 2; ++q) {  // 4 dims -> one 32-bit word of hi and of lo
+                    const float2 f0 = __bfloat1622float2(b2[2 * q]), f1 = __bfloat1622float2(b2[2 * q + 1]);
+                    const float x0 = f0.x * inv, x1 = f0.y * inv, x2 = f1.x * inv, x3 = f1.y * inv;
+                    const uint32_t h01 = ptx::e4m3x2(x0, x1), h23 = ptx::e4m3x2(x2, x3);
+                    float a0, a1, a2, a3;
+                    ptx::e4m3x2_to_f32(h01, &a0, &a1);
+                    ptx::e4m3x2_to_f32(h23, &a2, &a3);
+                    hw[2 * h + q] = h01 | (h23 << 16);
+                    lw[2 * h + q] = ptx::e4m3x2(x0 - a0, x1 - a1) | (ptx::e4m3x2(x2 - a2, x3 - a3) << 16);
                 }
             }
+            const uint4 hi4 = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            const uint4 lo4 = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             const int rl = row + kN;   // lo row
             if (uu < 32) {
                 const int c = uu >> 3, k = uu & 7;
@@ -455,16 +507,30 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
             }
         }
     } else {
-        for (int u = st; u < kN * 72; u += kSoftmaxThreads) {
-            const int row = u / 72, uu = u % 72;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (r0 + row < p.R) {
-                const __nv_bfloat16 *src = uu < 64 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 8
-                                                   : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 64) * 8;
-                v = __ldg(reinterpret_cast<const uint4 *>(src));
+        constexpr int kUnits = kN * 72;  // 8 dims per unit
+        constexpr int kPer = (kUnits + 2 * kSoftmaxThreads - 1) / (2 * kSoftmaxThreads);  // 7 per batch
+#pragma unroll 1
+        for (int batch = 0; batch < 2; ++batch) {
+            uint4 v[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int u = st + (batch * kPer + j) * kSoftmaxThreads;
+                const int row = u / 72, uu = u % 72;
+                v[j] = make_uint4(0, 0, 0, 0);
+                if (u < kUnits && r0 + row < p.R) {
+                    const __nv_bfloat16 *src = uu < 64 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 8
+                                                       : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 64) * 8;
+                    v[j] = __ldg(reinterpret_cast<const uint4 *>(src));
+                }
             }
-            const int c = uu >> 3, k = uu & 7;
-            *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4)) = v;
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int u = st + (batch * kPer + j) * kSoftmaxThreads;
+                if (u >= kUnits) continue;
+                const int row = u / 72, uu = u % 72;
+                const int c = uu >> 3, k = uu & 7;
+                *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4)) = v[j];
+            }
         }
     }
     return true;
@@ -558,8 +624,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         for (int k = 0; k < nt; ++k) {
             const uint32_t gg = g0 + k;
             const int stage = gg % C::kStages;
-            if (!waitb(p, ms, &ms.kv_full[stage], (gg / C::kStages) & 1)) return;
-            const uint32_t info = ms.stage_info[stage];
+            // part 0 carries the value scales; the tile's page mask was written before it
+            if (!waitb(p, ms, &ms.part_full[stage][0], (gg / C::kStages) & 1)) return;
+            const uint32_t info = ms.stage_info[gg & 3];
             piece_bad |= (info >> 31) != 0;
             const int sb = gg % C::kSBufs;
             if (!waitb(p, ms, &ms.s_full[sb], (gg / C::kSBufs) & 1)) return;
@@ -731,18 +798,24 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         }
         if (!hsync(p, ms)) return;
         const int ncols = min(kHalf, rows_here - cb);
+        // row c of this half, latent dim d = 128 m + i: consecutive lanes write
+        // consecutive dims of one row (coalesced); unrolled so o[] stays in registers
+        const int64_t row0 = pc.single ? (int64_t)pc.b * p.R + r0 + cb : (int64_t)pc.piece * p.R + r0 + cb;
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
             float o[kHalf];
             tmem_rows24<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
             const int d = 128 * m + i;
-            for (int c = 0; c < ncols; ++c) {
-                const float v = o[c] * ms.inv_l[cb + c];
-                const int64_t r = r0 + cb + c;
-                if (pc.single)
-                    store_out(p.out, ((int64_t)pc.b * p.R + r) * kDl + d, v, p.out_f32);
-                else
-                    p.part_o[((int64_t)pc.piece * p.R + r) * kDl + d] = v;
+#pragma unroll
+            for (int c = 0; c < kHalf; ++c) {
+                if (c < ncols) {
+                    const float v = o[c] * ms.inv_l[cb + c];
+                    const int64_t idx = (row0 + c) * kDl + d;
+                    if (pc.single)
+                        store_out(p.out, idx, v, p.out_f32);
+                    else
+                        p.part_o[idx] = v;
+                }
             }
         }
         if (hst < ncols) {
@@ -779,8 +852,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(&ms.kv_full[s], 1);
-            ptx::mbar_init(&ms.kv_empty[s], 1);
+            for (int q = 0; q < 9; ++q) {
+                ptx::mbar_init(&ms.part_full[s][q], 1);
+                ptx::mbar_init(&ms.part_empty[s][q], 1);
+            }
             ptx::mbar_init(&ms.s_full[s], 1);
             ptx::mbar_init(&ms.s_free[s], 8);
             ptx::mbar_init(&ms.half_sync[s], 4);
