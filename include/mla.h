@@ -92,7 +92,7 @@ typedef enum {
 } mla_device_error;
 
 typedef struct mla_dims {
-    int32_t B;                  /* sequences, >= 1 */
+    int32_t B;                  /* sequences, >= 1 (B*T*H <= 2^29 - 1) */
     int32_t T;                  /* query tokens per sequence (1 + drafts), 1..8 */
     int32_t H;                  /* query heads, >= 1 (T*H <= 1024) */
     int32_t num_pages;          /* P: pages in kv_pages */
@@ -103,9 +103,10 @@ typedef struct mla_dims {
     int32_t num_splits;         /* 0 = automatic; else number of KV ranges the pages are cut into */
     int32_t kernel;             /* mla_kernel */
     const int32_t *vis_lens;    /* device [B,T] visible positions per query token, or NULL */
-    void *stage_event;          /* optional cudaEvent_t, recorded on `stream` (as an external
-                                   event, so it also works inside graph capture) after the
-                                   attention kernel and before the merge kernel; NULL for none */
+    void *stage_event;          /* optional cudaEvent_t, recorded on `stream` after the
+                                   attention kernel and before the merge kernel (inside a stream
+                                   capture as an external event node, readable after each
+                                   replay); NULL for none */
 } mla_dims;
 
 /*
@@ -192,7 +193,7 @@ MLA_API int mla_decode_noalloc(const void *q_lat, const void *q_pe, const void *
  * L = max_i lse_i; w_i = exp(lse_i - L); out = sum_i w_i out_i / sum_i w_i;
  * lse = L + ln sum_i w_i.  Parts with lse = -inf weigh nothing; a row whose
  * parts are all -inf gets out = 0, lse = -inf; a NaN lse makes the row NaN.
- * 1 <= n_parts <= 4096, rows >= 0 (rows == 0 launches nothing).
+ * 1 <= n_parts <= 4096, 0 <= rows <= 2^29 - 1 (rows == 0 launches nothing).
  */
 MLA_API int mla_merge_partials(const float *out_parts, const float *lse_parts, int32_t n_parts,
                        int64_t rows, void *out, int32_t out_dtype, float *lse_out,

@@ -45,6 +45,7 @@ int check_dims(const mla_dims *d) {
     if (!d) return MLA_ERR_INVALID_ARG;
     if (d->B < 1 || d->T < 1 || d->T > kMaxT || d->H < 1 || (int64_t)d->T * d->H > kMaxRows)
         return MLA_ERR_INVALID_ARG;
+    if ((int64_t)d->B * d->T * d->H > ((int64_t)1 << 29) - 1) return MLA_ERR_INVALID_ARG;  // merge grid
     if (d->num_pages < 1 || d->max_pages_per_seq < 1 || d->page_table_stride < d->max_pages_per_seq)
         return MLA_ERR_INVALID_ARG;
     if (d->kv_dtype != MLA_KV_BF16 && d->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
@@ -152,8 +153,14 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     rc = pl.kernel == MLA_KERNEL_SIMT ? launch_simt(p, s) : launch_tc(p, s);
     if (rc) return rc;
     if (dims->stage_event) {
-        cudaError_t e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(dims->stage_event), s,
-                                                 cudaEventRecordExternal);
+        // inside a stream capture the record becomes an external event node
+        // (readable after each replay); outside one it is a plain record
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaError_t e = cudaStreamIsCapturing(s, &cs);
+        if (e == cudaSuccess)
+            e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(dims->stage_event), s,
+                                         cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                             : cudaEventRecordDefault);
         if (e != cudaSuccess) {
             note_cuda_error(e);
             return MLA_ERR_CUDA;
@@ -230,7 +237,7 @@ int mla_decode_noalloc(const void *q_lat, const void *q_pe, const void *kv_pages
 int mla_merge_partials(const float *out_parts, const float *lse_parts, int32_t n_parts, int64_t rows,
                        void *out, int32_t out_dtype, float *lse_out, mla_stream_t stream) {
     if (!out_parts || !lse_parts || !out) return MLA_ERR_INVALID_ARG;
-    if (n_parts < 1 || n_parts > 4096 || rows < 0 || rows > (int64_t)INT32_MAX) return MLA_ERR_INVALID_ARG;
+    if (n_parts < 1 || n_parts > 4096 || rows < 0 || rows > ((int64_t)1 << 29) - 1) return MLA_ERR_INVALID_ARG;
     if (out_dtype != MLA_OUT_BF16 && out_dtype != MLA_OUT_F32) return MLA_ERR_INVALID_ARG;
     if (!aligned(out_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16) ||
         (lse_out && !aligned(lse_out, 4)))

@@ -40,7 +40,7 @@
 // the e4m3 weights in range.  Row sums are kept per lane and reduced once per
 // piece.
 //
-// Every wait is bounded: after two seconds the CTA records a timeout in the
+// Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA records a timeout in the
 // error word, stops, drains its outstanding copies and MMAs and frees its
 // tensor memory.
 #include <cuda.h>
@@ -60,7 +60,7 @@ constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 soft
 constexpr int kSoftmaxThreads = 256;
 constexpr int kHalf = 24;              // query rows per softmax thread (two halves of 48)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kWaitLimit = 4000000000ull;  // SM cycles: about two seconds
 constexpr int kDevTimeout = 4;
 constexpr int kPrefetchAhead = 3;      // L2 prefetch distance, tiles
 
@@ -90,7 +90,7 @@ struct Cfg {
     static constexpr int kPGroupRows = kFp8 ? 16 : 8;
     static constexpr int kPBytes = (kNMma / kPGroupRows) * kTileM * 16;           // 12288 both
     static constexpr int kPLoOff = kFp8 ? (kN / 16) * kTileM * 16 : 0;             // lo rows start (group 3)
-    static constexpr int kMiscOff = kPOff + kPBytes;
+    static constexpr int kMiscOff = kPOff + 2 * kPBytes;                           // P double-buffered
     // Each stage is filled and freed in parts: the value chunks (FP8 4 x 128
     // dims, bf16 8 x 64 dims) and the RoPE chunk, so the next tile's copies
     // start as soon as the previous tile's MMAs are done with each part.
@@ -107,7 +107,8 @@ struct Cfg {
 struct Misc {
     uint64_t part_full[2][9], part_empty[2][9];   // per KV stage and part
     uint64_t s_full[2], s_free[2];
-    uint64_t p_full, pv_done, q_ready, o_free, drain;
+    uint64_t p_full[2], pv_done[2];  // per P buffer: weights written / value MMAs of that buffer done
+    uint64_t q_ready, o_free, drain;
     uint64_t all_sync;        // the eight softmax warps (bounded waits, unlike bar.sync)
     uint64_t half_sync[2];    // the four softmax warps of each row half
     uint32_t tmem_base;
@@ -136,7 +137,7 @@ __device__ __forceinline__ void cta_abort(const Problem &p, Misc &ms) {
 __device__ __forceinline__ bool aborted(Misc &ms) { return *reinterpret_cast<volatile int *>(&ms.abort) != 0; }
 
 __device__ __forceinline__ bool waitb(const Problem &p, Misc &ms, uint64_t *bar, uint32_t parity) {
-    if (ptx::mbar_wait(bar, parity, kWaitLimitNs)) return true;
+    if (ptx::mbar_wait(bar, parity, kWaitLimit)) return true;
     cta_abort(p, ms);
     return false;
 }
@@ -151,9 +152,23 @@ struct GroupSync {
     __device__ __forceinline__ bool operator()(const Problem &p, Misc &ms) {
         __syncwarp();
         if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
-        const bool ok = waitb(p, ms, bar, phase & 1);
+        // the other warps arrive within a few hundred cycles: poll without
+        // suspending, checking the clock every 64 polls
+        const uint32_t par = phase & 1;
         ++phase;
-        return ok;
+        uint64_t t0 = 0;
+        for (uint32_t i = 0;; ++i) {
+            if (ptx::mbar_test(bar, par)) return true;
+            if ((i & 63) == 63) {
+                const uint64_t t = ptx::cycles();
+                if (t0 == 0) {
+                    t0 = t;
+                } else if (t - t0 > kWaitLimit || aborted(ms)) {
+                    cta_abort(p, ms);
+                    return false;
+                }
+            }
+        }
     }
 };
 
@@ -173,14 +188,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Query split for the e4m3 score MMA: hi = e4m3(x), lo = e4m3(x - hi).
-__device__ __forceinline__ void split_e4m3(float x, uint8_t &hi, uint8_t &lo) {
-    const __nv_fp8_e4m3 h(x);              // round to nearest, saturating
-    const __nv_fp8_e4m3 l(x - float(h));
-    hi = h.__x;
-    lo = l.__x;
-}
-
 // ---------------------------------------------------------------------------
 // warp 0: TMA producer
 // ---------------------------------------------------------------------------
@@ -190,23 +197,18 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
     using C = Cfg<kFp8>;
     const int lane = threadIdx.x & 31;
     uint32_t g = 0;
-    // L2 warm-up of tile k of a piece: page ids, then one prefetch per page/box
+    // L2 warm-up of tile k of a piece: a page is one contiguous block of
+    // 16 x 576 elements, so one bulk prefetch per page (tensor-map prefetches
+    // would cost the copy engine one operation per box).
+    constexpr uint32_t kPageBytes = kFp8 ? kPage * kD : kPage * kD * 2;
     auto prefetch_tile = [&](const Piece &pc, int k) {
         const int pg0 = pc.page_lo + k * kTilePages;
         const int npg = min(kTilePages, pc.page_hi - pg0);
         if (npg <= 0 || lane >= npg) return;
         const int pid = __ldg(p.page_table + (int64_t)pc.b * p.pt_stride + pg0 + lane);
         if (pid < 0 || pid >= p.num_pages) return;
-        const int y = pid * kPage;
-        if constexpr (kFp8) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::tma_prefetch_2d(map_a, 128 * c, y);
-            ptx::tma_prefetch_2d(map_b, 512, y);
-            ptx::bulk_prefetch(p.kv_scale + (int64_t)pid * kPage, 64);
-        } else {
-#pragma unroll
-            for (int c = 0; c < 9; ++c) ptx::tma_prefetch_2d(map_a, 64 * c, y);
-        }
+        ptx::bulk_prefetch(static_cast<const unsigned char *>(p.kv) + (int64_t)pid * kPageBytes, kPageBytes);
+        if constexpr (kFp8) ptx::bulk_prefetch(p.kv_scale + (int64_t)pid * kPage, 64);
     };
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
@@ -259,7 +261,7 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
     // make sure no copy is still landing when the CTA leaves
     for (uint32_t h = g > (uint32_t)C::kStages ? g - C::kStages : 0; h < g; ++h)
         for (int part = 0; part < C::kParts; ++part)
-            ptx::mbar_wait(&ms.part_full[h % C::kStages][part], (h / C::kStages) & 1, kWaitLimitNs);
+            ptx::mbar_wait(&ms.part_full[h % C::kStages][part], (h / C::kStages) & 1, kWaitLimit);
 }
 
 // ---------------------------------------------------------------------------
@@ -279,59 +281,60 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                                        : ptx::instr_desc(1, 1, 1, 1, kTileM, C::kNMma);
     uint32_t g = 0, pi = 0;
 
+    // Shared-memory descriptors are built once; an MMA then only adds the
+    // byte offset of its operands (>> 4) to the start-address field.
+    constexpr uint64_t kStageStep = (uint64_t)(C::kStageBytes >> 4);
+    const uint64_t dq_kv = ptx::smem_desc(kv0, 16, 1024, ptx::kSwizzle128B);       // K-major 128B chunks
+    const uint64_t dq_q = ptx::smem_desc(q0, 16, 1024, ptx::kSwizzle128B);
+    const uint64_t dr_kv = ptx::smem_desc(kv0 + 4 * C::kChunkBytes, 16, 512, ptx::kSwizzle64B);  // FP8 RoPE
+    const uint64_t dr_q = ptx::smem_desc(q0 + C::kQRopeOff, 16, 512, ptx::kSwizzle64B);
+    const uint64_t dv_kv = ptx::smem_desc(kv0, 16384, 1024, ptx::kSwizzle128B);   // V^T, MN-major
+    const uint64_t dv_p = ptx::smem_desc(p0, 128, 2048, ptx::kSwizzleNone);       // P^T, MN-major
+
     // Score MMAs reading one part of the tile (accumulate from the second MMA of the tile on).
     auto issue_qk_part = [&](uint32_t gg, int part, bool first) {
-        const uint32_t st = kv0 + (gg % C::kStages) * C::kStageBytes;
+        const uint64_t so = (gg % C::kStages) * kStageStep;
         const uint32_t d = tmem + ((gg % C::kSBufs) ? C::kColS1 : 0u);
         if constexpr (kFp8) {
             // N = 96: query rows 0-47 hold hi, 48-95 hold lo
             if (part == C::kRope) {
 #pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    uint64_t a = ptx::smem_desc(st + 4 * C::kChunkBytes + ks * 32, 16, 512, ptx::kSwizzle64B);
-                    uint64_t b = ptx::smem_desc(q0 + C::kQRopeOff + ks * 32, 16, 512, ptx::kSwizzle64B);
-                    ptx::mma_f8(d, a, b, idesc_qk, (first && ks == 0) ? 0u : 1u);
-                }
+                for (int ks = 0; ks < 2; ++ks)
+                    ptx::mma_f8(d, dr_kv + so + 2 * ks, dr_q + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
             } else {
+                const uint64_t a = dq_kv + so + part * (C::kChunkBytes >> 4);
+                const uint64_t b = dq_q + part * (C::kQChunk >> 4);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    uint64_t a = ptx::smem_desc(st + part * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                    uint64_t b = ptx::smem_desc(q0 + part * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                    ptx::mma_f8(d, a, b, idesc_qk, (first && ks == 0) ? 0u : 1u);
-                }
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::mma_f8(d, a + 2 * ks, b + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
             }
         } else {
+            const uint64_t a = dq_kv + so + part * (C::kChunkBytes >> 4);
+            const uint64_t b = dq_q + part * (C::kQChunk >> 4);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                uint64_t a = ptx::smem_desc(st + part * C::kChunkBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                uint64_t b = ptx::smem_desc(q0 + part * C::kQChunk + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                ptx::mma_f16(d, a, b, idesc_qk, (first && ks == 0) ? 0u : 1u);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+                ptx::mma_f16(d, a + 2 * ks, b + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
         }
     };
 
     // Value MMAs; each 128-dim block frees its value chunk(s) of the stage as it completes.
     auto issue_pv = [&](uint32_t gg, bool first) {
         const int stage = gg % C::kStages;
-        const uint32_t st = kv0 + stage * C::kStageBytes;
+        const uint64_t a0 = dv_kv + stage * kStageStep;
+        const uint64_t pb = dv_p + (gg & 1) * (uint64_t)(C::kPBytes >> 4);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const uint32_t d = tmem + C::kColO + C::kOStride * m;
             if constexpr (kFp8) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {  // 32 positions per MMA; N = 96: P hi | P lo
-                    uint64_t a = ptx::smem_desc(st + m * C::kChunkBytes + ks * 4096, 16384, 1024, ptx::kSwizzle128B);
-                    uint64_t b = ptx::smem_desc(p0 + ks * 512, 128, 2048, ptx::kSwizzleNone);
-                    ptx::mma_f8(d, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
-                }
+                for (int ks = 0; ks < 4; ++ks)  // 32 positions per MMA; N = 96: P hi | P lo
+                    ptx::mma_f8(d, a0 + m * (C::kChunkBytes >> 4) + ks * (4096 >> 4), pb + ks * (512 >> 4),
+                                idesc_pv, (first && ks == 0) ? 0u : 1u);
             } else {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {  // 16 positions per MMA
-                    uint64_t a = ptx::smem_desc(st + 2 * m * C::kChunkBytes + ks * 2048, 16384, 1024,
-                                                ptx::kSwizzle128B);
-                    uint64_t b = ptx::smem_desc(p0 + ks * 256, 128, 2048, ptx::kSwizzleNone);
-                    ptx::mma_f16(d, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
-                }
+                for (int ks = 0; ks < 8; ++ks)  // 16 positions per MMA
+                    ptx::mma_f16(d, a0 + 2 * m * (C::kChunkBytes >> 4) + ks * (2048 >> 4), pb + ks * (256 >> 4),
+                                 idesc_pv, (first && ks == 0) ? 0u : 1u);
             }
             if constexpr (kFp8) {
                 ptx::mma_commit(&ms.part_empty[stage][m]);
@@ -342,70 +345,81 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
         }
     };
 
-    // Barrier tests are made by lane 0 and broadcast, so the warp never diverges
-    // on a phase that completes while it polls.
-    auto test = [&](uint64_t *bar, uint32_t parity) -> bool {
-        const int r = lane == 0 ? (int)ptx::mbar_test(bar, parity) : 0;
-        return __shfl_sync(0xffffffffu, r, 0) != 0;
+    // Waits are made by lane 0 and broadcast, so the warp never diverges on
+    // a phase that completes (or a limit that expires) while it waits.
+    auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {
+        int ok = 1;
+        if (lane == 0) ok = ptx::mbar_wait(bar, parity, kWaitLimit) && !aborted(ms);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) cta_abort(p, ms);
+        return ok != 0;
     };
 
+    // Two groups per tile k: the scores of tile k (all its parts landed and
+    // the score buffer free) and the values of tile k - 1 (its weights
+    // written).  Lane 0 polls both and the warp issues whichever is ready
+    // first; the values go first when both are, since they free the stage
+    // that the next copy waits for.
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
         if (nt == 0 || aborted(ms)) return;
         const uint32_t g0 = g;
-        int nq = 0, qp = 0, npv = 0;   // tiles whose scores / values are issued; parts of tile nq issued
-        bool q_ok = false, o_ok = false, s_ok = false;
-        uint64_t t_idle = ptx::globaltimer();
-        // Issue each MMA group as soon as its operands are ready: the values of
-        // tile k as soon as its weights are written (each value block then
-        // frees its chunk for the next copy), the scores of tile k part by part
-        // as the parts land.
-        while (npv < nt) {
-            bool progress = false;
-            if (npv < nq) {
-                const uint32_t gp = g0 + npv;
-                if (!o_ok && npv == 0) o_ok = test(&ms.o_free, (pi & 1) ^ 1);
-                if ((npv > 0 || o_ok) && test(&ms.p_full, gp & 1)) {
-                    ptx::tc_fence_after();
-                    if (lane == 0) {
-                        issue_pv(gp, npv == 0);
-                        ptx::mma_commit(&ms.pv_done);
-                    }
-                    __syncwarp();
-                    ++npv;
-                    progress = true;
+        if (!wait1(&ms.q_ready, pi & 1)) return;
+        int nq = 0, nv = 0;        // score / value groups issued
+        int qp = 0;                // parts of tile nq seen landed
+        bool s_ok = false, o_ok = false;
+        uint64_t t_idle = ptx::cycles();
+        uint32_t spins = 0;
+        while (nv < nt) {
+            // lane 0 decides; 1 = values, 2 = scores, 0 = nothing ready yet
+            int pick = 0;
+            if (lane == 0) {
+                if (nv < nq) {
+                    const uint32_t gp = g0 + nv;
+                    if (nv == 0 && !o_ok) o_ok = ptx::mbar_test(&ms.o_free, (pi & 1) ^ 1);
+                    if ((nv > 0 || o_ok) && ptx::mbar_test(&ms.p_full[gp & 1], (gp >> 1) & 1)) pick = 1;
+                }
+                if (pick == 0 && nq < nt && nq <= nv + 1) {
+                    const uint32_t gq = g0 + nq;
+                    const int stage = gq % C::kStages;
+                    if (!s_ok) s_ok = ptx::mbar_test(&ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1);
+                    while (s_ok && qp < C::kParts &&
+                           ptx::mbar_test(&ms.part_full[stage][qp == 0 ? C::kRope : qp - 1], (gq / C::kStages) & 1))
+                        ++qp;
+                    if (s_ok && qp == C::kParts) pick = 2;
                 }
             }
-            if (nq < nt) {
+            pick = __shfl_sync(0xffffffffu, pick, 0);
+            if (pick == 1) {
+                const uint32_t gp = g0 + nv;
+                ptx::tc_fence_after();
+                if (lane == 0) {
+                    issue_pv(gp, nv == 0);
+                    ptx::mma_commit(&ms.pv_done[gp & 1]);
+                }
+                __syncwarp();
+                ++nv;
+            } else if (pick == 2) {
                 const uint32_t gq = g0 + nq;
                 const int stage = gq % C::kStages;
-                if (!q_ok) q_ok = test(&ms.q_ready, pi & 1);
-                if (q_ok && qp == 0 && !s_ok) s_ok = test(&ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1);
-                while (q_ok && s_ok && qp < C::kParts) {
-                    const int part = qp == 0 ? C::kRope : qp - 1;
-                    if (!test(&ms.part_full[stage][part], (gq / C::kStages) & 1)) break;
-                    ptx::tc_fence_after();
-                    if (lane == 0) issue_qk_part(gq, part, qp == 0);
-                    __syncwarp();
-                    ++qp;
-                    progress = true;
+                ptx::tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int q = 0; q < C::kParts; ++q) issue_qk_part(gq, q == 0 ? C::kRope : q - 1, q == 0);
+                    ptx::mma_commit(&ms.s_full[gq % C::kSBufs]);
+                    ptx::mma_commit(&ms.part_empty[stage][C::kRope]);  // RoPE is read by scores only
                 }
-                if (qp == C::kParts) {
-                    if (lane == 0) {
-                        ptx::mma_commit(&ms.s_full[gq % C::kSBufs]);
-                        ptx::mma_commit(&ms.part_empty[stage][C::kRope]);  // RoPE is read by scores only
-                    }
-                    __syncwarp();
-                    ++nq;
-                    qp = 0;
-                    s_ok = false;
-                }
+                __syncwarp();
+                ++nq;
+                qp = 0;
+                s_ok = false;
             }
-            if (progress) {
-                if (lane == 0) t_idle = ptx::globaltimer();
-            } else {
+            if (pick != 0) {
+                t_idle = ptx::cycles();
+                spins = 0;
+            } else if ((++spins & 255) == 0) {
                 int expired = 0;
-                if (lane == 0) expired = (ptx::globaltimer() - t_idle > kWaitLimitNs) || aborted(ms);
+                if (lane == 0) expired = (ptx::cycles() - t_idle > kWaitLimit) || aborted(ms);
                 if (__shfl_sync(0xffffffffu, expired, 0)) {
                     cta_abort(p, ms);
                     return;
@@ -418,7 +432,7 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
     // every MMA issued has completed before tensor memory is released
     if (lane == 0) ptx::mma_commit(&ms.drain);
     __syncwarp();
-    ptx::mbar_wait(&ms.drain, 0, kWaitLimitNs);
+    ptx::mbar_wait(&ms.drain, 0, kWaitLimit);
 }
 
 // ---------------------------------------------------------------------------
@@ -442,6 +456,7 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
         constexpr int kPer = (kUnits + kSoftmaxThreads - 1) / kSoftmaxThreads;  // 7
         uint4 v[kPer][2];
         float amax = 0.f;
+        // every load is issued before any is used: one memory round trip
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int u = st + j * kSoftmaxThreads;
@@ -453,6 +468,9 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
                 v[j][0] = __ldg(reinterpret_cast<const uint4 *>(src));
                 v[j][1] = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
             }
+        }
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v[j][h]);
@@ -636,6 +654,8 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&ms.s_free[sb]);
+            // P buffer gg & 1 is free once the value MMAs of tile gg - 2 are done
+            if (gg >= 2 && !waitb(p, ms, &ms.pv_done[gg & 1], ((gg - 2) >> 1) & 1)) return;
 
             const int pos0 = (pc.page_lo + k * kTilePages) * kPage;
             const int pos = pos0 + i;
@@ -686,7 +706,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 if (!hsync(p, ms)) return;  // red[] reads done before any reuse
                 if (moved && k > 0) {
                     // O^T holds earlier tiles: wait for their value MMA, then rescale rows
-                    if (!waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
+                    if (!waitb(p, ms, &ms.pv_done[(gg - 1) & 1], ((gg - 1) >> 1) & 1)) return;
                     ptx::tc_fence_after();
 #pragma unroll 1
                     for (int m = 0; m < 4; ++m) {
@@ -721,9 +741,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     for (int e = 0; e < 8; ++e) row[e] = make_uint4(0, 0, 0, 0);
                 }
             }
-            // the single P buffer is free once the previous tile's value MMA is done
-            if (gg > 0 && !waitb(p, ms, &ms.pv_done, (gg - 1) & 1)) return;
-            unsigned char *pb = smem + C::kPOff;
+            unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
             if constexpr (kFp8) {
                 // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of the half
                 uint32_t hw[kHalf / 4], lw[kHalf / 4];
@@ -771,12 +789,13 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&ms.p_full);
+            if (lane == 0) ptx::mbar_arrive(&ms.p_full[gg & 1]);
         }
         g = g0 + nt;
 
         // ---- epilogue: row sums, normalised output, log-sum-exp
-        if (!waitb(p, ms, &ms.pv_done, (g - 1) & 1)) return;
+        // the last value MMAs done (a commit covers every earlier MMA too)
+        if (!waitb(p, ms, &ms.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) return;
         ptx::tc_fence_after();
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) {
@@ -801,6 +820,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         // row c of this half, latent dim d = 128 m + i: consecutive lanes write
         // consecutive dims of one row (coalesced); unrolled so o[] stays in registers
         const int64_t row0 = pc.single ? (int64_t)pc.b * p.R + r0 + cb : (int64_t)pc.piece * p.R + r0 + cb;
+        float inv_l[kHalf];
+#pragma unroll
+        for (int c = 0; c < kHalf; ++c) inv_l[c] = ms.inv_l[cb + c];
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
             float o[kHalf];
@@ -809,7 +831,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
 #pragma unroll
             for (int c = 0; c < kHalf; ++c) {
                 if (c < ncols) {
-                    const float v = o[c] * ms.inv_l[cb + c];
+                    const float v = o[c] * inv_l[c];
                     const int64_t idx = (row0 + c) * kDl + d;
                     if (pc.single)
                         store_out(p.out, idx, v, p.out_f32);
@@ -860,8 +882,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&ms.s_free[s], 8);
             ptx::mbar_init(&ms.half_sync[s], 4);
         }
-        ptx::mbar_init(&ms.p_full, 8);
-        ptx::mbar_init(&ms.pv_done, 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&ms.p_full[b], 8);
+            ptx::mbar_init(&ms.pv_done[b], 1);
+        }
         ptx::mbar_init(&ms.q_ready, 8);
         ptx::mbar_init(&ms.o_free, 8);
         ptx::mbar_init(&ms.drain, 1);

@@ -14,9 +14,12 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
+// SM cycle counter: cheap to read, used to bound waits.  (The global
+// nanosecond timer costs hundreds of cycles per read, which would sit on the
+// critical path of every polling loop.)
+__device__ __forceinline__ uint64_t cycles() {
     uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
     return t;
 }
 
@@ -65,13 +68,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// `limit_ns` nanoseconds and returns false, so that no wait can hang.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+// `limit_cycles` SM cycles and returns false, so that no wait can hang.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_cycles) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+    const uint64_t t0 = cycles();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > limit_ns) return false;
+        if (cycles() - t0 > limit_cycles) return false;
     }
 }
 
