@@ -69,6 +69,39 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = ("mla_latent_attention_b200/csrc/mla_tc.cu", "mla_latent_attention_b200/csrc/mla_common.cuh",
+                  "mla_latent_attention_b200/csrc/tc_ptx.cuh")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kv: str):
+    """DRAM bytes per launch of the attention kernel from an ncu capture,
+    recorded in profiles/ncu_traffic.txt as
+    ``<workload> <kv> <kernel source hash> <dram read+write bytes per launch>``.
+    None when there is no capture for the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    try:
+        with open(path) as f:
+            lines = f.read().splitlines()
+    except OSError:
+        return None
+    want = kernel_source_hash()
+    for ln in lines:
+        parts = ln.split()
+        if len(parts) == 4 and not ln.startswith("#") and parts[0] == workload and parts[1] == kv \
+                and parts[2] == want:
+            return float(parts[3])
+    return None
+
+
 def visible_positions(w) -> int:
     """Sum over query rows' distinct sequences of cached positions read once
     per layer (each sequence's pages are read once for all its rows)."""
@@ -370,7 +403,8 @@ def run_ours(args, rank, world, local_rank):
     achieved_gbs = per_launch_bytes / dec_avg / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak, "traffic": None,
+                "frac": achieved_gbs / hbm_peak, "traffic": recorded_traffic(args.workload, w.kv_dtype),
+                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "kernel": "mla decode attention kernel", "peak_source": f"{peak_src} hbm_gbs",
                 "avg_launch_us": dec_avg * 1e6, "merge_avg_launch_us": sum(mer) / len(mer) * 1e6}
     tflops = per_launch_flops / dec_avg / 1e12

@@ -136,6 +136,7 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     p.err = reinterpret_cast<int32_t *>(ws);
     p.part_lse = reinterpret_cast<float *>(ws + pl.lse_off);
     p.part_o = reinterpret_cast<float *>(ws + pl.o_off);
+    p.max_pieces = pl.max_pieces;
     p.B = dims->B;
     p.T = dims->T;
     p.H = dims->H;

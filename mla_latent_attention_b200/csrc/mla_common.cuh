@@ -29,8 +29,13 @@ struct Problem {
     const int32_t *vis_lens;      // [B,T] or null
     void *out;                    // [B,T,H,512]
     float *lse;                   // [B,T,H] or null
-    float *part_o;                // [pieces,R,512] normalised partial outputs
-    float *part_lse;              // [pieces,R]
+    // split-KV partials, row-major over pieces: the pieces of one query row
+    // sit next to each other, so the merge reads each row's parts as one
+    // contiguous run (no large power-of-two stride that lands every part of a
+    // row in the same cache slices)
+    float *part_o;                // [R, max_pieces, 512] normalised partial outputs
+    float *part_lse;              // [R, max_pieces]
+    int64_t max_pieces;           // piece stride of the partials
     int32_t *err;                 // workspace error word {code, info}
     int B, T, H, R;               // R = T*H query rows per sequence
     int num_pages, max_pages, pt_stride;

@@ -6,163 +6,194 @@
 //   L = max_i lse_i,  w_i = exp(lse_i - L),
 //   out = sum_i w_i out_i / sum_i w_i,  lse = L + ln sum_i w_i.
 //
-// One CTA per (output row, quarter of the 512 latent dims), 256 threads:
-// thread (grp, c) = (tid / 32, tid % 32) accumulates dims 128q + 4c .. +3
-// over the parts i = grp (mod 8), four parts in flight at a time; the eight
-// groups are then summed through shared memory.  Rows x 4 CTAs keep every
-// SM streaming even when a single sequence has few query rows.
+// Work unit = (output row, quarter of the 512 latent dims): 32 lanes x 4 dims.
+// Each lane combines its parts online, one pass over them:
+//   m <- max(m, lse_i);  s, acc rescaled by exp(m_old - m);  then += w_i, w_i out_i
+// which is the formula above with L replaced by a running maximum.  Loads are
+// issued eight parts at a time before any is used.
+//   * few parts: one warp per unit, eight units per CTA;
+//   * many parts: one CTA per unit, eight warps each taking every eighth part,
+//     their (m, s, acc) then combined through shared memory.
 #include "mla_common.cuh"
 
 namespace mla {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kGroups = kThreads / 32;
+constexpr int kWarps = kThreads / 32;
 constexpr int kQuarters = 4;
+constexpr int kFewParts = 16;
+constexpr int kBatch = 8;     // parts in flight per lane, one warp per unit
+constexpr int kCtaBatch = 8;  // the same, eight warps per unit
 
-struct MergeSmem {
-    float4 acc[kGroups - 1][32];
-    float wsum[kGroups];
-    float red[kGroups];
-    int nan_flag;
+struct Online {
+    float m = -INFINITY, s = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    bool nan = false;
 };
 
-// parts i of this row: out at o0 + i*o_stride, lse at l0 + i*l_stride.
-__device__ __forceinline__ void merge_row(const float *o0, int64_t o_stride, const float *l0,
-                                          int64_t l_stride, int n, void *out, int64_t out_row,
-                                          int out_f32, float *lse_out, int quarter, MergeSmem &sm) {
-    const int tid = threadIdx.x, c = tid & 31, grp = tid >> 5;
-    // 1) max lse, NaN detection
-    float L = -INFINITY;
-    int has_nan = 0;
-    for (int i = tid; i < n; i += kThreads) {
-        const float l = __ldg(l0 + i * l_stride);
-        if (isnan(l)) has_nan = 1;
-        L = fmaxf(L, l);
-    }
+// parts first, first + step, ... < n of one unit: lse at l0[i*l_stride], the
+// lane's four dims at v0[i*v_stride] (float4 units)
+template <int kB>
+__device__ __forceinline__ void combine_parts(Online &st, const float *l0, int64_t l_stride, const float4 *v0,
+                                              int64_t v_stride, int first, int step, int n) {
+    for (int base = first; base < n; base += kB * step) {
+        float l[kB];
+        float4 v[kB];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
-    has_nan = __any_sync(0xffffffffu, has_nan);
-    if (tid == 0) sm.nan_flag = 0;
-    __syncthreads();
-    if (c == 0) {
-        sm.red[grp] = L;
-        if (has_nan) sm.nan_flag = 1;
-    }
-    __syncthreads();
-    L = sm.red[0];
-#pragma unroll
-    for (int w = 1; w < kGroups; ++w) L = fmaxf(L, sm.red[w]);
-    const bool nan_row = sm.nan_flag != 0;
-
-    // 2) weighted sums, parts strided over the groups
-    const float4 *v0 = reinterpret_cast<const float4 *>(o0) + quarter * 32 + c;
-    const int64_t v_stride = o_stride / 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float wsum = 0.f;
-    if (!nan_row && L != -INFINITY) {
-        int i = grp;
-        for (; i + 3 * kGroups < n; i += 4 * kGroups) {
-            float w[4];
-            float4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int k = i + u * kGroups;
-                w[u] = __ldg(l0 + k * l_stride);
-                v[u] = __ldg(v0 + k * v_stride);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                // a part that saw nothing weighs nothing, whatever its out holds
-                const bool empty = w[u] == -INFINITY;
-                const float ww = empty ? 0.f : expf(w[u] - L);
-                if (empty) v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                wsum += ww;
-                acc.x = fmaf(ww, v[u].x, acc.x);
-                acc.y = fmaf(ww, v[u].y, acc.y);
-                acc.z = fmaf(ww, v[u].z, acc.z);
-                acc.w = fmaf(ww, v[u].w, acc.w);
+        for (int u = 0; u < kB; ++u) {
+            const int i = base + u * step;
+            l[u] = -INFINITY;
+            if (i < n) {
+                l[u] = __ldg(l0 + i * l_stride);
+                v[u] = __ldg(v0 + i * v_stride);
             }
         }
-        for (; i < n; i += kGroups) {
-            const float l = __ldg(l0 + i * l_stride);
-            if (l == -INFINITY) continue;
-            const float ww = expf(l - L);
-            const float4 v = __ldg(v0 + i * v_stride);
-            wsum += ww;
-            acc.x = fmaf(ww, v.x, acc.x);
-            acc.y = fmaf(ww, v.y, acc.y);
-            acc.z = fmaf(ww, v.z, acc.z);
-            acc.w = fmaf(ww, v.w, acc.w);
-        }
-    }
-    if (grp > 0) sm.acc[grp - 1][c] = acc;
-    if (c == 0) sm.wsum[grp] = wsum;
-    __syncthreads();
-    if (grp == 0) {
-        float W = sm.wsum[0];
 #pragma unroll
-        for (int g2 = 1; g2 < kGroups; ++g2) {
-            const float4 a = sm.acc[g2 - 1][c];
-            acc.x += a.x;
-            acc.y += a.y;
-            acc.z += a.z;
-            acc.w += a.w;
-            W += sm.wsum[g2];
+        for (int u = 0; u < kB; ++u) {
+            if (isnan(l[u])) st.nan = true;
+            // a part that saw nothing weighs nothing, whatever its out holds
+            if (!(l[u] > -INFINITY)) continue;
+            if (l[u] > st.m) {
+                const float sc = __expf(st.m - l[u]);  // m = -inf -> 0
+                st.s *= sc;
+                st.acc.x *= sc;
+                st.acc.y *= sc;
+                st.acc.z *= sc;
+                st.acc.w *= sc;
+                st.m = l[u];
+            }
+            const float w = __expf(l[u] - st.m);
+            st.s += w;
+            st.acc.x = fmaf(w, v[u].x, st.acc.x);
+            st.acc.y = fmaf(w, v[u].y, st.acc.y);
+            st.acc.z = fmaf(w, v[u].z, st.acc.z);
+            st.acc.w = fmaf(w, v[u].w, st.acc.w);
         }
-        float4 o;
-        float lse;
-        if (nan_row) {
-            o = make_float4(NAN, NAN, NAN, NAN);
-            lse = NAN;
-        } else if (L == -INFINITY) {
-            o = make_float4(0.f, 0.f, 0.f, 0.f);
-            lse = -INFINITY;
-        } else {
-            const float inv = 1.f / W;
-            o = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-            lse = L + logf(W);
-        }
-        const int64_t base = out_row * kDl + 128 * quarter + 4 * c;
-        if (out_f32) {
-            reinterpret_cast<float4 *>(static_cast<float *>(out) + base)[0] = o;
-        } else {
-            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(o.x, o.y);
-            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(o.z, o.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t *>(&lo2);
-            pk.y = *reinterpret_cast<const uint32_t *>(&hi2);
-            reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + base)[0] = pk;
-        }
-        if (c == 0 && quarter == 0 && lse_out) lse_out[out_row] = lse;
     }
 }
 
+__device__ __forceinline__ void write_unit(const Online &st, void *out, int64_t out_row, int quarter, int lane,
+                                           int out_f32, float *lse_out) {
+    float4 o;
+    float lse;
+    if (st.nan) {
+        o = make_float4(NAN, NAN, NAN, NAN);
+        lse = NAN;
+    } else if (!(st.s > 0.f)) {
+        o = make_float4(0.f, 0.f, 0.f, 0.f);
+        lse = -INFINITY;
+    } else {
+        const float inv = 1.f / st.s;
+        o = make_float4(st.acc.x * inv, st.acc.y * inv, st.acc.z * inv, st.acc.w * inv);
+        lse = st.m + logf(st.s);
+    }
+    const int64_t base = out_row * kDl + 128 * quarter + 4 * lane;
+    if (out_f32) {
+        reinterpret_cast<float4 *>(static_cast<float *>(out) + base)[0] = o;
+    } else {
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(o.x, o.y);
+        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(o.z, o.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t *>(&lo2);
+        pk.y = *reinterpret_cast<const uint32_t *>(&hi2);
+        reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + base)[0] = pk;
+    }
+    if (lane == 0 && quarter == 0 && lse_out) lse_out[out_row] = lse;
+}
+
+struct MergeSmem {
+    float4 acc[kWarps][32];
+    float m[kWarps], s[kWarps];
+    int nan[kWarps];
+};
+
+// One unit, all eight warps of the CTA over its parts (many parts).
+__device__ __forceinline__ void merge_unit_cta(const float *o0, int64_t o_stride, const float *l0, int64_t l_stride,
+                                               int n, void *out, int64_t out_row, int quarter, int out_f32,
+                                               float *lse_out, MergeSmem &sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    Online st;
+    combine_parts<kCtaBatch>(st, l0, l_stride, reinterpret_cast<const float4 *>(o0) + quarter * 32 + lane, o_stride / 4,
+                             warp, kWarps, n);
+    sm.acc[warp][lane] = st.acc;
+    if (lane == 0) {
+        sm.m[warp] = st.m;
+        sm.s[warp] = st.s;
+        sm.nan[warp] = st.nan;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        Online t;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) t.m = fmaxf(t.m, sm.m[w]);
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            t.nan |= sm.nan[w] != 0;
+            if (!(sm.s[w] > 0.f)) continue;
+            const float sc = __expf(sm.m[w] - t.m);
+            const float4 a = sm.acc[w][lane];
+            t.s = fmaf(sc, sm.s[w], t.s);
+            t.acc.x = fmaf(sc, a.x, t.acc.x);
+            t.acc.y = fmaf(sc, a.y, t.acc.y);
+            t.acc.z = fmaf(sc, a.z, t.acc.z);
+            t.acc.w = fmaf(sc, a.w, t.acc.w);
+        }
+        write_unit(t, out, out_row, quarter, lane, out_f32, lse_out);
+    }
+}
+
+// One unit per warp (few parts).
+__device__ __forceinline__ void merge_unit_warp(const float *o0, int64_t o_stride, const float *l0, int64_t l_stride,
+                                                int n, void *out, int64_t out_row, int quarter, int out_f32,
+                                                float *lse_out) {
+    const int lane = threadIdx.x & 31;
+    Online st;
+    combine_parts<kBatch>(st, l0, l_stride, reinterpret_cast<const float4 *>(o0) + quarter * 32 + lane, o_stride / 4, 0,
+                          1, n);
+    write_unit(st, out, out_row, quarter, lane, out_f32, lse_out);
+}
+
 // Rows of sequences that were split into several pieces by mla_decode.
-__global__ void __launch_bounds__(kThreads) merge_internal_kernel(Problem p) {
+// kCta: one unit per CTA (many pieces), else one unit per warp.
+// three unit-CTAs per SM: a row set of one sequence (96 rows x 4 quarters) is one wave
+template <bool kCta>
+__global__ void __launch_bounds__(kThreads, kCta ? 3 : 1) merge_internal_kernel(Problem p) {
     __shared__ MergeSmem sm;
-    const int64_t grow = blockIdx.x / kQuarters;  // b * R + r
-    const int quarter = blockIdx.x % kQuarters;
+    const int64_t unit = kCta ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t grow = unit / kQuarters;  // b * R + r
+    if (grow >= (int64_t)p.B * p.R) return;
+    const int quarter = (int)(unit % kQuarters);
     const int b = (int)(grow / p.R), r = (int)(grow % p.R);
     int n_pieces = 0, piece_base = 0;
     bool bad = false;
     pieces_of(p, b, &n_pieces, &piece_base, &bad);
     if (n_pieces < 2) return;  // finished by the decode kernel
-    const float *o0 = p.part_o + ((int64_t)piece_base * p.R + r) * kDl;
-    const float *l0 = p.part_lse + (int64_t)piece_base * p.R + r;
-    merge_row(o0, (int64_t)p.R * kDl, l0, p.R, n_pieces, p.out, grow, p.out_f32, p.lse, quarter, sm);
+    // the pieces of row r are contiguous: [r][piece][512]
+    const float *o0 = p.part_o + ((int64_t)r * p.max_pieces + piece_base) * kDl;
+    const float *l0 = p.part_lse + (int64_t)r * p.max_pieces + piece_base;
+    if (kCta)
+        merge_unit_cta(o0, kDl, l0, 1, n_pieces, p.out, grow, quarter, p.out_f32, p.lse, sm);
+    else
+        merge_unit_warp(o0, kDl, l0, 1, n_pieces, p.out, grow, quarter, p.out_f32, p.lse);
 }
 
 // mla_merge_partials: parts laid out [n_parts, rows, 512] and [n_parts, rows].
-__global__ void __launch_bounds__(kThreads) merge_public_kernel(const float *out_parts,
-                                                                const float *lse_parts, int n_parts,
-                                                                int64_t rows, void *out, int out_f32,
+template <bool kCta>
+__global__ void __launch_bounds__(kThreads, kCta ? 3 : 1) merge_public_kernel(const float *out_parts, const float *lse_parts,
+                                                                int n_parts, int64_t rows, void *out, int out_f32,
                                                                 float *lse_out) {
     __shared__ MergeSmem sm;
-    const int64_t row = blockIdx.x / kQuarters;
-    const int quarter = blockIdx.x % kQuarters;
-    merge_row(out_parts + row * kDl, rows * kDl, lse_parts + row, rows, n_parts, out, row, out_f32,
-              lse_out, quarter, sm);
+    const int64_t unit = kCta ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int64_t row = unit / kQuarters;
+    if (row >= rows) return;
+    const int quarter = (int)(unit % kQuarters);
+    if (kCta)
+        merge_unit_cta(out_parts + row * kDl, rows * kDl, lse_parts + row, rows, n_parts, out, row, quarter, out_f32,
+                       lse_out, sm);
+    else
+        merge_unit_warp(out_parts + row * kDl, rows * kDl, lse_parts + row, rows, n_parts, out, row, quarter,
+                        out_f32, lse_out);
 }
 
 }  // namespace
@@ -170,7 +201,15 @@ __global__ void __launch_bounds__(kThreads) merge_public_kernel(const float *out
 int launch_merge_internal(const Problem &p, cudaStream_t stream) {
     const int64_t rows = (int64_t)p.B * p.R;
     if (rows <= 0) return MLA_OK;
-    merge_internal_kernel<<<(unsigned)(rows * kQuarters), kThreads, 0, stream>>>(p);
+    // Slots much more numerous than sequences mean many pieces per sequence:
+    // eight warps per unit.  Otherwise a warp per unit (it handles any number
+    // of pieces, only more slowly when there are many).
+    const bool many = p.n_slots > 2 * p.B;
+    const int64_t units = rows * kQuarters;
+    if (many)
+        merge_internal_kernel<true><<<(unsigned)units, kThreads, 0, stream>>>(p);
+    else
+        merge_internal_kernel<false><<<(unsigned)((units + kWarps - 1) / kWarps), kThreads, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         note_cuda_error(e);
@@ -182,8 +221,13 @@ int launch_merge_internal(const Problem &p, cudaStream_t stream) {
 int launch_merge_public(const float *out_parts, const float *lse_parts, int n_parts, int64_t rows,
                         void *out, int out_f32, float *lse_out, cudaStream_t stream) {
     if (rows == 0) return MLA_OK;
-    merge_public_kernel<<<(unsigned)(rows * kQuarters), kThreads, 0, stream>>>(out_parts, lse_parts, n_parts,
-                                                                               rows, out, out_f32, lse_out);
+    const int64_t units = rows * kQuarters;
+    if (n_parts > kFewParts)
+        merge_public_kernel<true><<<(unsigned)units, kThreads, 0, stream>>>(out_parts, lse_parts, n_parts, rows, out,
+                                                                           out_f32, lse_out);
+    else
+        merge_public_kernel<false><<<(unsigned)((units + kWarps - 1) / kWarps), kThreads, 0, stream>>>(
+            out_parts, lse_parts, n_parts, rows, out, out_f32, lse_out);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         note_cuda_error(e);

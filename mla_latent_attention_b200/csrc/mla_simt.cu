@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(Problem p) {
                 store_out(p.out, grow * kDl + d0 + 1, o1, p.out_f32);
                 if (tid == 0 && p.lse) p.lse[grow] = lse;
             } else {
-                int64_t prow = (int64_t)pc.piece * p.R + r;
+                int64_t prow = (int64_t)r * p.max_pieces + pc.piece;
                 p.part_o[prow * kDl + d0] = o0;
                 p.part_o[prow * kDl + d0 + 1] = o1;
                 if (tid == 0) p.part_lse[prow] = lse;

@@ -152,23 +152,9 @@ struct GroupSync {
     __device__ __forceinline__ bool operator()(const Problem &p, Misc &ms) {
         __syncwarp();
         if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
-        // the other warps arrive within a few hundred cycles: poll without
-        // suspending, checking the clock every 64 polls
-        const uint32_t par = phase & 1;
+        const bool ok = waitb(p, ms, bar, phase & 1);
         ++phase;
-        uint64_t t0 = 0;
-        for (uint32_t i = 0;; ++i) {
-            if (ptx::mbar_test(bar, par)) return true;
-            if ((i & 63) == 63) {
-                const uint64_t t = ptx::cycles();
-                if (t0 == 0) {
-                    t0 = t;
-                } else if (t - t0 > kWaitLimit || aborted(ms)) {
-                    cta_abort(p, ms);
-                    return false;
-                }
-            }
-        }
+        return ok;
     }
 };
 
@@ -417,7 +403,10 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
             if (pick != 0) {
                 t_idle = ptx::cycles();
                 spins = 0;
-            } else if ((++spins & 255) == 0) {
+            } else if ((++spins & 3) == 0) {
+                __nanosleep(32);  // leave issue slots to the softmax warps of this scheduler
+            }
+            if (pick == 0 && (spins & 255) == 0) {
                 int expired = 0;
                 if (lane == 0) expired = (ptx::cycles() - t_idle > kWaitLimit) || aborted(ms);
                 if (__shfl_sync(0xffffffffu, expired, 0)) {
@@ -743,18 +732,19 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             }
             unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
             if constexpr (kFp8) {
-                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of the half
+                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of the
+                // half.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
+                // far below lo's 2^-9), hi = e4m3(p16), and p16 - hi is exact in
+                // f16, so lo = e4m3(p16 - hi).
                 uint32_t hw[kHalf / 4], lw[kHalf / 4];
 #pragma unroll
                 for (int w = 0; w < kHalf / 4; ++w) {
                     uint32_t hp[2], lp[2];
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
-                        const float a = s[4 * w + 2 * q], b = s[4 * w + 2 * q + 1];
-                        hp[q] = ptx::e4m3x2(a, b);
-                        float fa, fb;
-                        ptx::e4m3x2_to_f32(hp[q], &fa, &fb);
-                        lp[q] = ptx::e4m3x2(a - fa, b - fb);
+                        const uint32_t p16 = ptx::f16x2(s[4 * w + 2 * q], s[4 * w + 2 * q + 1]);
+                        hp[q] = ptx::e4m3x2_from_f16x2(p16);
+                        lp[q] = ptx::e4m3x2_from_f16x2(ptx::sub_f16x2(p16, ptx::f16x2_from_e4m3x2(hp[q])));
                     }
                     hw[w] = hp[0] | (hp[1] << 16);
                     lw[w] = lp[0] | (lp[1] << 16);
@@ -819,7 +809,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         const int ncols = min(kHalf, rows_here - cb);
         // row c of this half, latent dim d = 128 m + i: consecutive lanes write
         // consecutive dims of one row (coalesced); unrolled so o[] stays in registers
-        const int64_t row0 = pc.single ? (int64_t)pc.b * p.R + r0 + cb : (int64_t)pc.piece * p.R + r0 + cb;
+        // output row c: out[b*R + r] (whole sequence) or the partial [r][piece]
+        const int64_t row0 = pc.single ? (int64_t)pc.b * p.R + r0 + cb : (int64_t)(r0 + cb) * p.max_pieces + pc.piece;
+        const int64_t row_step = pc.single ? 1 : p.max_pieces;
         float inv_l[kHalf];
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) inv_l[c] = ms.inv_l[cb + c];
@@ -832,7 +824,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             for (int c = 0; c < kHalf; ++c) {
                 if (c < ncols) {
                     const float v = o[c] * inv_l[c];
-                    const int64_t idx = (row0 + c) * kDl + d;
+                    const int64_t idx = (row0 + c * row_step) * kDl + d;
                     if (pc.single)
                         store_out(p.out, idx, v, p.out_f32);
                     else
@@ -845,7 +837,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             if (pc.single) {
                 if (p.lse) p.lse[(int64_t)pc.b * p.R + r] = ms.lse[cb + hst];
             } else {
-                p.part_lse[(int64_t)pc.piece * p.R + r] = ms.lse[cb + hst];
+                p.part_lse[r * p.max_pieces + pc.piece] = ms.lse[cb + hst];
             }
         }
         ptx::tc_fence_before();

@@ -282,6 +282,33 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t v, float *x0, float *x1) 
     *x1 = b;
 }
 
+// Two floats -> f16x2 (round to nearest): x0 in the low half.
+__device__ __forceinline__ uint32_t f16x2(float x0, float x1) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(x1), "f"(x0));
+    return r;
+}
+
+// f16x2 -> two e4m3 bytes (round to nearest even, saturating), order kept.
+__device__ __forceinline__ uint32_t e4m3x2_from_f16x2(uint32_t h) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h));
+    return r;
+}
+
+// Two e4m3 bytes -> f16x2 (exact), order kept.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t v) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}" : "=r"(h2) : "r"(v));
+    return h2;
+}
+
+__device__ __forceinline__ uint32_t sub_f16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
