@@ -557,7 +557,8 @@ __device__ __forceinline__ void tmem_rows24(uint32_t taddr, float *v) {
 }
 
 template <bool kFp8>
-__device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, int slot, int g_idx) {
+__device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, int slot, int g_idx,
+                             const CUtensorMap *map_out, const CUtensorMap *map_part) {
     using C = Cfg<kFp8>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int w8 = warp - 2;                   // 0..7
@@ -807,31 +808,44 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         }
         if (!hsync(p, ms)) return;
         const int ncols = min(kHalf, rows_here - cb);
-        // row c of this half, latent dim d = 128 m + i: consecutive lanes write
-        // consecutive dims of one row (coalesced); unrolled so o[] stays in registers
-        // output row c: out[b*R + r] (whole sequence) or the partial [r][piece]
-        const int64_t row0 = pc.single ? (int64_t)pc.b * p.R + r0 + cb : (int64_t)(r0 + cb) * p.max_pieces + pc.piece;
-        const int64_t row_step = pc.single ? 1 : p.max_pieces;
+        // O goes out one 128-dim block at a time: every thread writes its dim of
+        // its half's rows into a [48 rows][128] staging box (the query area is
+        // free until the next piece), then one thread stores the box with a
+        // tensor store.  The maps clip rows past the sequence's R, and two
+        // staging boxes alternate so the next block is written while the
+        // previous one is copied out.
         float inv_l[kHalf];
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) inv_l[c] = ms.inv_l[cb + c];
-#pragma unroll 1
+        const bool f32_box = !pc.single || p.out_f32;
+        constexpr int kBoxBytes = kN * 128 * 4;
         for (int m = 0; m < 4; ++m) {
+            unsigned char *box = smem + C::kQOff + (m & 1) * kBoxBytes;
+            if (m >= 2) {  // the store of block m - 2 has finished reading this box
+                if (st == 0) ptx::bulk_wait_read<1>();
+                if (!all_sync(p, ms)) return;
+            }
             float o[kHalf];
             tmem_rows24<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
-            const int d = 128 * m + i;
 #pragma unroll
             for (int c = 0; c < kHalf; ++c) {
-                if (c < ncols) {
-                    const float v = o[c] * inv_l[c];
-                    const int64_t idx = (row0 + c * row_step) * kDl + d;
-                    if (pc.single)
-                        store_out(p.out, idx, v, p.out_f32);
-                    else
-                        p.part_o[idx] = v;
-                }
+                const float v = o[c] * inv_l[c];
+                if (f32_box)
+                    reinterpret_cast<float *>(box)[(cb + c) * 128 + i] = v;
+                else
+                    reinterpret_cast<__nv_bfloat16 *>(box)[(cb + c) * 128 + i] = __float2bfloat16_rn(v);
+            }
+            ptx::fence_proxy_async_smem();
+            if (!all_sync(p, ms)) return;
+            if (st == 0) {
+                if (pc.single)
+                    ptx::tma_store_3d(map_out, box, 128 * m, r0, pc.b);
+                else
+                    ptx::tma_store_3d(map_part, box, 128 * m, (int)pc.piece, r0);
+                ptx::bulk_commit();
             }
         }
+        if (st == 0) ptx::bulk_wait_read<0>();  // boxes read before the query area is reused
         if (hst < ncols) {
             const int64_t r = r0 + cb + hst;
             if (pc.single) {
@@ -850,7 +864,8 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const __grid_constant__ Problem p, const __grid_constant__ CUtensorMap map_a,
-                     const __grid_constant__ CUtensorMap map_b) {
+                     const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_out,
+                     const __grid_constant__ CUtensorMap map_part) {
     using C = Cfg<kFp8>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -902,7 +917,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     else if (warp == 1)
         mma_issuer<kFp8>(p, smem, ms, slot);
     else
-        softmax_role<kFp8>(p, smem, ms, slot, g_idx);
+        softmax_role<kFp8>(p, smem, ms, slot, g_idx, &map_out, &map_part);
 
     ptx::tc_fence_before();
     __syncthreads();
@@ -941,9 +956,37 @@ bool make_kv_map(CUtensorMap *map, const void *base, int num_pages, bool fp8, ui
     return r == CUDA_SUCCESS;
 }
 
+// Output views for the epilogue's tensor stores, boxes of 128 dims x 48 rows:
+// out as [B][R][512] (bf16 or fp32), the partials as [R][pieces][512] fp32.
+bool make_out_maps(CUtensorMap *mo, CUtensorMap *mp, const Problem &p) {
+    auto encode = get_encode_fn();
+    if (!encode) return false;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const size_t osz = p.out_f32 ? 4 : 2;
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)p.R, (cuuint64_t)p.B};
+        const cuuint64_t strides[2] = {(cuuint64_t)kDl * osz, (cuuint64_t)p.R * kDl * osz};
+        const cuuint32_t box[3] = {128, (cuuint32_t)kN, 1};
+        if (encode(mo, p.out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.out, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    if (p.max_pieces < 1 || !p.part_o) {  // no partials: never stored through
+        *mp = *mo;
+        return true;
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)p.max_pieces, (cuuint64_t)p.R};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDl * 4, (cuuint64_t)p.max_pieces * kDl * 4};
+    const cuuint32_t box[3] = {128, 1, (cuuint32_t)kN};
+    return encode(mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.part_o, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool kFp8>
 int launch_impl(const Problem &p, cudaStream_t stream) {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mo, mp;
     bool ok;
     if (kFp8) {
         ok = make_kv_map(&ma, p.kv, p.num_pages, true, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -952,11 +995,12 @@ int launch_impl(const Problem &p, cudaStream_t stream) {
         ok = make_kv_map(&ma, p.kv, p.num_pages, false, 64, CU_TENSOR_MAP_SWIZZLE_128B);
         mb = ma;
     }
+    ok = ok && make_out_maps(&mo, &mp, p);
     if (!ok) return MLA_ERR_CUDA;
     const int smem = smem_bytes<kFp8>();
     cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess) {
-        tc_decode_kernel<kFp8><<<p.n_slots * p.n_groups, kThreads, smem, stream>>>(p, ma, mb);
+        tc_decode_kernel<kFp8><<<p.n_slots * p.n_groups, kThreads, smem, stream>>>(p, ma, mb, mo, mp);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) {
@@ -967,6 +1011,8 @@ int launch_impl(const Problem &p, cudaStream_t stream) {
 }
 
 static_assert(smem_bytes<true>() <= 232448, "FP8 tile does not fit shared memory");
+static_assert(2 * kN * 128 * 4 <= Cfg<true>::kQBytes && 2 * kN * 128 * 4 <= Cfg<false>::kQBytes,
+              "two epilogue staging boxes must fit the query area");
 static_assert(smem_bytes<false>() <= 232448, "bf16 tile does not fit shared memory");
 static_assert(Cfg<true>::kColO + 3 * Cfg<true>::kOStride + Cfg<true>::kNMma <= kTmemCols, "TMEM overflow");
 static_assert(Cfg<false>::kColO + 3 * Cfg<false>::kOStride + Cfg<false>::kNMma <= kTmemCols, "TMEM overflow");
