@@ -62,7 +62,6 @@ constexpr int kHalf = 24;              // query rows per softmax thread (two hal
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 4000000000ull;  // SM cycles: about two seconds
 constexpr int kDevTimeout = 4;
-constexpr int kPrefetchAhead = 3;      // L2 prefetch distance, tiles
 
 template <bool kFp8>
 struct Cfg {
@@ -183,24 +182,15 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
     using C = Cfg<kFp8>;
     const int lane = threadIdx.x & 31;
     uint32_t g = 0;
-    // L2 warm-up of tile k of a piece: a page is one contiguous block of
-    // 16 x 576 elements, so one bulk prefetch per page (tensor-map prefetches
-    // would cost the copy engine one operation per box).
-    constexpr uint32_t kPageBytes = kFp8 ? kPage * kD : kPage * kD * 2;
-    auto prefetch_tile = [&](const Piece &pc, int k) {
-        const int pg0 = pc.page_lo + k * kTilePages;
-        const int npg = min(kTilePages, pc.page_hi - pg0);
-        if (npg <= 0 || lane >= npg) return;
-        const int pid = __ldg(p.page_table + (int64_t)pc.b * p.pt_stride + pg0 + lane);
-        if (pid < 0 || pid >= p.num_pages) return;
-        ptx::bulk_prefetch(static_cast<const unsigned char *>(p.kv) + (int64_t)pid * kPageBytes, kPageBytes);
-        if constexpr (kFp8) ptx::bulk_prefetch(p.kv_scale + (int64_t)pid * kPage, 64);
-    };
+    bool first_piece = true;
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
-        for (int k = 1; k < min(nt, kPrefetchAhead); ++k) prefetch_tile(pc, k);
         for (int k = 0; k < nt; ++k, ++g) {
             if (aborted(ms)) return;
+            // At launch every CTA wants its first tiles and its query at once;
+            // the second tile waits until the query is staged, so that the
+            // query's bytes are not queued behind tile copies.
+            if (first_piece && k == 1 && !waitb(p, ms, &ms.q_ready, 0)) return;
             const int stage = g % C::kStages;
             const uint32_t empty_parity = ((g / C::kStages) & 1) ^ 1;
             const int pg0 = pc.page_lo + k * kTilePages;
@@ -241,8 +231,8 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                     ptx::tma_load_2d(st + part * C::kChunkBytes + lane * 2048, map_a, bar, 64 * part, y);
                 }
             }
-            if (k + kPrefetchAhead < nt) prefetch_tile(pc, k + kPrefetchAhead);
         }
+        first_piece = false;
     });
     // make sure no copy is still landing when the CTA leaves
     for (uint32_t h = g > (uint32_t)C::kStages ? g - C::kStages : 0; h < g; ++h)
