@@ -35,9 +35,10 @@
 // Softmax stabiliser: per query row a running bound m2 on the log2 weight
 // u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
 // the lanes of a row half.  It moves only when some weight exceeds it by more
-// than TAU (then O^T and the row sums are rescaled), which after the first
-// tile is rare.  Weights are exp2(u - m2 + C), at most 2^(TAU+C), which keeps
-// the e4m3 weights in range.  Row sums are kept per lane and reduced once per
+// than TAU (then O^T and the row sums are rescaled), and then to DELTA above
+// the new maximum, so after the first tile it rarely moves again.  Weights
+// are exp2(u - m2 + C), at most 2^(TAU+C), which keeps the e4m3 weights in
+// range.  Row sums are kept per lane and reduced once per
 // piece.
 //
 // Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA records a timeout in the
@@ -98,9 +99,13 @@ struct Cfg {
     __host__ __device__ static constexpr uint32_t part_bytes(int part) {            // per page
         return kFp8 ? (part == kRope ? 1024u : (part == 0 ? 2048u + 64u : 2048u)) : 2048u;
     }
-    // exponent offset C and lazy threshold TAU of the softmax stabiliser
+    // exponent offset C and lazy threshold TAU of the softmax stabiliser, and
+    // the headroom DELTA it is placed above a new maximum when it moves (so
+    // that later, slightly larger scores do not move it again at once); the
+    // largest weight stays below 2^(C + TAU) either way.
     static constexpr float kC = kFp8 ? 4.5f : 0.f;
     static constexpr float kTau = kFp8 ? 4.f : 8.f;
+    static constexpr float kDelta = kFp8 ? 2.f : 0.f;
 };
 
 struct Misc {
@@ -677,7 +682,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     const float cm = fmaxf(fmaxf(ms.red[h][0][c], ms.red[h][1][c]),
                                            fmaxf(ms.red[h][2][c], ms.red[h][3][c]));
                     const float old = m2c[c] + C::kC;
-                    const float mn = cm > old + C::kTau ? cm : old;
+                    const float mn = cm > old + C::kTau ? cm + C::kDelta : old;
                     alpha[c] = mn == old ? 1.f : ptx::ex2(old - mn);
                     moved |= mn != old;
                     m2c[c] = mn - C::kC;
