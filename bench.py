@@ -74,11 +74,17 @@ KERNEL_SOURCES = ("mla_latent_attention_b200/csrc/mla_tc.cu", "mla_latent_attent
 
 
 def kernel_source_hash() -> str:
+    """Hash of the attention kernel's sources with comments and blank space
+    removed, so that editing a comment does not orphan a recorded capture."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

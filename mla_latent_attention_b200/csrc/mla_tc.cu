@@ -26,11 +26,13 @@
 //     adds the two halves of O^T.  V is read as stored, never dequantised.
 // bf16 caches use kind::f16 MMAs with N = 48 and bf16 P.
 //
-// Warp roles (320 threads): warp 0 issues TMA page loads (and warms L2 with
-// the tiles after them), warp 1 issues the MMAs -- each as soon as its
-// operands are ready -- and owns tensor memory, warps 2-9 run the online
-// softmax and the epilogue.  Thread (warp w, lane l) owns tile position /
-// TMEM lane 32*(w%4) + l; warps 2-5 take query rows 0-23, warps 6-9 rows 24-47.
+// Warp roles (448 threads): warp 0 issues TMA page loads, warp 1 issues the
+// MMAs -- each group as soon as its operands are ready -- and owns tensor
+// memory, warps 2-13 run the online softmax and the epilogue.  Thread
+// (warp w, lane l) owns tile position / TMEM lane 32*(w%4) + l; the softmax
+// warps form three groups of four (one per TMEM lane quadrant), each group
+// taking 16 of the 48 query rows.  (Fourteen warps leave 128 registers per
+// thread; sixteen softmax warps of 12 rows would leave 96 and spill.)
 //
 // Softmax stabiliser: per query row a running bound m2 on the log2 weight
 // u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
@@ -57,9 +59,11 @@ namespace {
 constexpr int kN = 48;                 // query rows per CTA
 constexpr int kTileM = 128;            // positions per tile (MMA M)
 constexpr int kTilePages = kTileM / kPage;
-constexpr int kThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
-constexpr int kSoftmaxThreads = 256;
-constexpr int kHalf = 24;              // query rows per softmax thread (two halves of 48)
+constexpr int kRowGroups = 3;                       // softmax warp sets, one per 16 of the 48 rows
+constexpr int kSoftmaxWarps = 4 * kRowGroups;       // x 4 TMEM lane quadrants
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kThreads = 64 + kSoftmaxThreads;      // warp 0 TMA, warp 1 MMA, warps 2.. softmax
+constexpr int kRpt = kN / kRowGroups;               // query rows per softmax thread
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 4000000000ull;  // SM cycles: about two seconds
 constexpr int kDevTimeout = 4;
@@ -113,17 +117,17 @@ struct Misc {
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], pv_done[2];  // per P buffer: weights written / value MMAs of that buffer done
     uint64_t q_ready, o_free, drain;
-    uint64_t all_sync;        // the eight softmax warps (bounded waits, unlike bar.sync)
-    uint64_t half_sync[2];    // the four softmax warps of each row half
+    uint64_t all_sync;        // all softmax warps (bounded waits, unlike bar.sync)
+    uint64_t half_sync[kRowGroups];  // the four softmax warps of each row group
     uint32_t tmem_base;
     int abort;
     uint32_t stage_info[4];   // per tile mod 4: bit i page slot i loaded; bit 31 a page was invalid
-    int vote[2][2][4];        // [half][tile parity][warp]
+    int vote[kRowGroups][2][4];  // [row group][tile parity][warp]
     int col_lim[kN];          // positions visible to row r within this piece, 0 = none
     int col_bad[kN];
     float qscale;
-    float amax[8];
-    float red[2][4][kHalf];   // [half][warp][row]
+    float amax[kSoftmaxWarps];
+    float red[kRowGroups][4][kRpt];  // [row group][warp][row]
     float m2c[kN];
     float inv_l[kN];
     float lse[kN];
@@ -469,7 +473,7 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
         if ((threadIdx.x & 31) == 0) ms.amax[(threadIdx.x >> 5) - 2] = amax;
         if (!gsync(p, ms)) return false;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) amax = fmaxf(amax, ms.amax[w]);
+        for (int w = 0; w < kSoftmaxWarps; ++w) amax = fmaxf(amax, ms.amax[w]);
         int e2 = 0;
         if (amax > 0.f) frexpf(amax / 448.f, &e2);
         const float inv = ldexpf(1.f, -e2);
@@ -541,13 +545,13 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
 // 24 rows of one accumulator column block; for FP8 the hi and lo halves
 // (48 columns apart) are added.
 template <bool kFp8>
-__device__ __forceinline__ void tmem_rows24(uint32_t taddr, float *v) {
-    ptx::tmem_ld24(taddr, v);
+__device__ __forceinline__ void tmem_rows(uint32_t taddr, float *v) {
+    ptx::tmem_ld_cols<kRpt>(taddr, v);
     if constexpr (kFp8) {
-        float w[kHalf];
-        ptx::tmem_ld24(taddr + kN, w);
+        float w[kRpt];
+        ptx::tmem_ld_cols<kRpt>(taddr + kN, w);
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c) v[c] += w[c];
+        for (int c = 0; c < kRpt; ++c) v[c] += w[c];
     }
 }
 
@@ -556,14 +560,14 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                              const CUtensorMap *map_out, const CUtensorMap *map_part) {
     using C = Cfg<kFp8>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int w8 = warp - 2;                   // 0..7
-    const int h = w8 >> 2;                     // row half: rows [24h, 24h + 24)
-    const int w4 = w8 & 3;                     // warp within the half
+    const int ws = warp - 2;                   // softmax warp 0 .. kSoftmaxWarps - 1
+    const int h = ws >> 2;                     // row group: rows [kRpt h, kRpt (h + 1))
+    const int w4 = ws & 3;                     // warp within the row group
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int i = quad * 32 + lane;            // tile position / TMEM lane
     const int st = threadIdx.x - 64;           // 0..255 for cooperative loops
-    const int hst = w4 * 32 + lane;            // 0..127 within the half
-    const int cb = h * kHalf;
+    const int hst = w4 * 32 + lane;            // 0..127 within the row group
+    const int cb = h * kRpt;
     const uint32_t tmem = ms.tmem_base + ((uint32_t)(quad * 32) << 16);
     const int r0 = g_idx * kN;
     constexpr float kEmpty = -1e30f;           // stabiliser of a row that has seen nothing yet
@@ -595,7 +599,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (!all_sync(p, ms)) return;
         const int rows_here = min(kN, p.R - r0);
         int min_lim = INT_MAX;  // over this half's real rows
-        for (int c = cb; c < min(cb + kHalf, rows_here); ++c) min_lim = min(min_lim, ms.col_lim[c]);
+        for (int c = cb; c < min(cb + kRpt, rows_here); ++c) min_lim = min(min_lim, ms.col_lim[c]);
 
         if (nt == 0) {  // nothing to read: write the empty (or invalid) result
             for (int e = st; e < rows_here * kDl; e += kSoftmaxThreads) {
@@ -616,9 +620,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         const float qscale = kFp8 ? ms.qscale : 1.f;
 
         // m2c = stabiliser - C: weights are ex2(score - m2c)
-        float m2c[kHalf], lsum[kHalf];
+        float m2c[kRpt], lsum[kRpt];
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c) {
+        for (int c = 0; c < kRpt; ++c) {
             m2c[c] = kEmpty;
             lsum[c] = 0.f;
         }
@@ -634,8 +638,8 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             const int sb = gg % C::kSBufs;
             if (!waitb(p, ms, &ms.s_full[sb], (gg / C::kSBufs) & 1)) return;
             ptx::tc_fence_after();
-            float s[kHalf];
-            tmem_rows24<kFp8>(tmem + (sb ? C::kColS1 : 0u) + cb, s);
+            float s[kRpt];
+            tmem_rows<kFp8>(tmem + (sb ? C::kColS1 : 0u) + cb, s);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&ms.s_free[sb]);
@@ -658,7 +662,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             const float kx = C::kC + C::kTau - lkvs;
             bool exceed = false;
 #pragma unroll
-            for (int c = 0; c < kHalf; ++c) {
+            for (int c = 0; c < kRpt; ++c) {
                 const bool valid = fast || (loaded && pos < ms.col_lim[cb + c]);
                 s[c] = valid ? s[c] * factor : -INFINITY;       // score, log2 units
                 exceed |= s[c] > m2c[c] + kx;
@@ -670,15 +674,15 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             const int *vv = ms.vote[h][gg & 1];
             if (vv[0] | vv[1] | vv[2] | vv[3]) {
 #pragma unroll
-                for (int c = 0; c < kHalf; ++c) {
+                for (int c = 0; c < kRpt; ++c) {
                     const float cm = warp_max(s[c] + lkvs);
                     if (lane == 0) ms.red[h][w4][c] = cm;
                 }
                 if (!hsync(p, ms)) return;
-                float alpha[kHalf];
+                float alpha[kRpt];
                 bool moved = false;
 #pragma unroll
-                for (int c = 0; c < kHalf; ++c) {
+                for (int c = 0; c < kRpt; ++c) {
                     const float cm = fmaxf(fmaxf(ms.red[h][0][c], ms.red[h][1][c]),
                                            fmaxf(ms.red[h][2][c], ms.red[h][3][c]));
                     const float old = m2c[c] + C::kC;
@@ -697,12 +701,12 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     for (int m = 0; m < 4; ++m) {
 #pragma unroll 1
                         for (int part = 0; part < (kFp8 ? 2 : 1); ++part) {
-                            float o[kHalf];
+                            float o[kRpt];
                             const uint32_t oc = tmem + C::kColO + C::kOStride * m + part * kN + cb;
-                            ptx::tmem_ld24(oc, o);
+                            ptx::tmem_ld_cols<kRpt>(oc, o);
 #pragma unroll
-                            for (int c = 0; c < kHalf; ++c) o[c] *= alpha[c];
-                            ptx::tmem_st24(oc, o);
+                            for (int c = 0; c < kRpt; ++c) o[c] *= alpha[c];
+                            ptx::tmem_st_cols<kRpt>(oc, o);
                         }
                     }
                 }
@@ -710,7 +714,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             // weights e = ex2(s - m2c) enter the row sums; the value MMA takes
             // e times the token's value scale (FP8) as its P entry
 #pragma unroll
-            for (int c = 0; c < kHalf; ++c) {
+            for (int c = 0; c < kRpt; ++c) {
                 const float e = ptx::ex2(s[c] - m2c[c]);
                 lsum[c] += e;
                 s[c] = kFp8 ? e * kvs : e;
@@ -732,9 +736,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 // half.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
                 // far below lo's 2^-9), hi = e4m3(p16), and p16 - hi is exact in
                 // f16, so lo = e4m3(p16 - hi).
-                uint32_t hw[kHalf / 4], lw[kHalf / 4];
+                uint32_t hw[kRpt / 4], lw[kRpt / 4];
 #pragma unroll
-                for (int w = 0; w < kHalf / 4; ++w) {
+                for (int w = 0; w < kRpt / 4; ++w) {
                     uint32_t hp[2], lp[2];
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
@@ -745,31 +749,23 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     hw[w] = hp[0] | (hp[1] << 16);
                     lw[w] = lp[0] | (lp[1] << 16);
                 }
-                // 16-row groups: half 0 owns group 0 and the low 8 bytes of group 1,
-                // half 1 the high 8 bytes of group 1 and group 2 (lo: groups 3-5)
-                if (h == 0) {
-                    *reinterpret_cast<uint4 *>(pb + i * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint2 *>(pb + 2048 + i * 16) = make_uint2(hw[4], hw[5]);
-                    *reinterpret_cast<uint4 *>(pb + C::kPLoOff + i * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                    *reinterpret_cast<uint2 *>(pb + C::kPLoOff + 2048 + i * 16) = make_uint2(lw[4], lw[5]);
-                } else {
-                    *reinterpret_cast<uint2 *>(pb + 2048 + i * 16 + 8) = make_uint2(hw[0], hw[1]);
-                    *reinterpret_cast<uint4 *>(pb + 4096 + i * 16) = make_uint4(hw[2], hw[3], hw[4], hw[5]);
-                    *reinterpret_cast<uint2 *>(pb + C::kPLoOff + 2048 + i * 16 + 8) = make_uint2(lw[0], lw[1]);
-                    *reinterpret_cast<uint4 *>(pb + C::kPLoOff + 4096 + i * 16) =
-                        make_uint4(lw[2], lw[3], lw[4], lw[5]);
+                // P^T is [16-row groups of 16 B] x 128 positions; each four of this
+                // thread's rows lie in one group
+#pragma unroll
+                for (int w = 0; w < kRpt / 4; ++w) {
+                    const int row0 = cb + 4 * w;
+                    const int off = (row0 >> 4) * 2048 + i * 16 + (row0 & 15);
+                    *reinterpret_cast<uint32_t *>(pb + off) = hw[w];
+                    *reinterpret_cast<uint32_t *>(pb + C::kPLoOff + off) = lw[w];
                 }
             } else {
+                // bf16 P^T: [8-row groups of 16 B] x 128 positions, two rows per word
 #pragma unroll
-                for (int j = 0; j < 3; ++j) {
-                    uint32_t wv[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(s[8 * j + 2 * q], s[8 * j + 2 * q + 1]);
-                        wv[q] = *reinterpret_cast<uint32_t *>(&b2);
-                    }
-                    *reinterpret_cast<uint4 *>(pb + (3 * h + j) * 2048 + i * 16) =
-                        make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                for (int w = 0; w < kRpt / 2; ++w) {
+                    const int row0 = cb + 2 * w;
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(s[2 * w], s[2 * w + 1]);
+                    *reinterpret_cast<uint32_t *>(pb + (row0 >> 3) * 2048 + i * 16 + 2 * (row0 & 7)) =
+                        *reinterpret_cast<uint32_t *>(&b2);
                 }
             }
             ptx::fence_proxy_async_smem();
@@ -784,16 +780,16 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (!waitb(p, ms, &ms.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) return;
         ptx::tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c) {
+        for (int c = 0; c < kRpt; ++c) {
             const float v = warp_sum(lsum[c]);
             if (lane == 0) ms.red[h][w4][c] = v;
         }
         if (hst == 0) {
 #pragma unroll
-            for (int c = 0; c < kHalf; ++c) ms.m2c[cb + c] = m2c[c];
+            for (int c = 0; c < kRpt; ++c) ms.m2c[cb + c] = m2c[c];
         }
         if (!hsync(p, ms)) return;
-        if (hst < kHalf) {
+        if (hst < kRpt) {
             const int col = cb + hst;
             const float l = ms.red[h][0][hst] + ms.red[h][1][hst] + ms.red[h][2][hst] + ms.red[h][3][hst];
             const bool bad = piece_bad || ms.col_bad[col];
@@ -802,16 +798,16 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             ms.lse[col] = bad ? NAN : (l > 0.f ? (ms.m2c[col] + __log2f(l)) * kLn2 : -INFINITY);
         }
         if (!hsync(p, ms)) return;
-        const int ncols = min(kHalf, rows_here - cb);
+        const int ncols = min(kRpt, rows_here - cb);
         // O goes out one 128-dim block at a time: every thread writes its dim of
         // its half's rows into a [48 rows][128] staging box (the query area is
         // free until the next piece), then one thread stores the box with a
         // tensor store.  The maps clip rows past the sequence's R, and two
         // staging boxes alternate so the next block is written while the
         // previous one is copied out.
-        float inv_l[kHalf];
+        float inv_l[kRpt];
 #pragma unroll
-        for (int c = 0; c < kHalf; ++c) inv_l[c] = ms.inv_l[cb + c];
+        for (int c = 0; c < kRpt; ++c) inv_l[c] = ms.inv_l[cb + c];
         const bool f32_box = !pc.single || p.out_f32;
         constexpr int kBoxBytes = kN * 128 * 4;
         for (int m = 0; m < 4; ++m) {
@@ -820,10 +816,10 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 if (st == 0) ptx::bulk_wait_read<1>();
                 if (!all_sync(p, ms)) return;
             }
-            float o[kHalf];
-            tmem_rows24<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
+            float o[kRpt];
+            tmem_rows<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
 #pragma unroll
-            for (int c = 0; c < kHalf; ++c) {
+            for (int c = 0; c < kRpt; ++c) {
                 const float v = o[c] * inv_l[c];
                 if (f32_box)
                     reinterpret_cast<float *>(box)[(cb + c) * 128 + i] = v;
@@ -881,17 +877,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_init(&ms.part_empty[s][q], 1);
             }
             ptx::mbar_init(&ms.s_full[s], 1);
-            ptx::mbar_init(&ms.s_free[s], 8);
-            ptx::mbar_init(&ms.half_sync[s], 4);
+            ptx::mbar_init(&ms.s_free[s], kSoftmaxWarps);
         }
+        for (int r = 0; r < kRowGroups; ++r) ptx::mbar_init(&ms.half_sync[r], 4);
         for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(&ms.p_full[b], 8);
+            ptx::mbar_init(&ms.p_full[b], kSoftmaxWarps);
             ptx::mbar_init(&ms.pv_done[b], 1);
         }
-        ptx::mbar_init(&ms.q_ready, 8);
-        ptx::mbar_init(&ms.o_free, 8);
+        ptx::mbar_init(&ms.q_ready, kSoftmaxWarps);
+        ptx::mbar_init(&ms.o_free, kSoftmaxWarps);
         ptx::mbar_init(&ms.drain, 1);
-        ptx::mbar_init(&ms.all_sync, 8);
+        ptx::mbar_init(&ms.all_sync, kSoftmaxWarps);
         ms.abort = 0;
         ptx::fence_mbar_init();
     }

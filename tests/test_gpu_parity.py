@@ -141,9 +141,11 @@ def test_context_partitions_merge_to_whole(kernel):
     assert (mo.float() - whole_o.float()).abs().max().item() <= 2e-2 * whole_o.float().abs().max().item()
 
 
-def test_merge_partials_matches_oracle():
+# 7 parts: one warp per (row, quarter); 40 parts: eight warps per (row, quarter)
+@pytest.mark.parametrize("n", [7, 40])
+def test_merge_partials_matches_oracle(n):
     gen = torch.Generator().manual_seed(3)
-    n, rows = 7, 37
+    rows = 37
     o = torch.randn((n, rows, 512), generator=gen, dtype=torch.float64)
     l = torch.randn((n, rows), generator=gen, dtype=torch.float64) * 3
     l[2, :5] = -float("inf")
@@ -209,6 +211,20 @@ def test_host_argument_errors_raise():
     with pytest.raises(mla.MlaError):
         mla.decode(w.q_lat, w.q_pe, w.kv_pages, None, w.page_table, w.ctx_lens, w.sm_scale,
                    workspace=torch.empty(16, dtype=torch.uint8, device=DEV))
+
+
+def test_stage_event_outside_capture():
+    """The optional stage event is a plain record when the stream is not being captured."""
+    w = W.make_workload("spec_verify_small", B=2).to(DEV)
+    ev = torch.cuda.Event()
+    ev.record()                  # torch creates the event handle on first record
+    torch.cuda.synchronize()
+    out, lse = mla.decode_workload(w, stage_event=ev)
+    torch.cuda.synchronize()
+    assert ev.query()
+    ref_o, ref_l = mla.decode_workload(w)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
