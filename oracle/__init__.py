@@ -65,6 +65,13 @@ def _bind(lib):
     lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
     lib.oracle_bf16_to_f64.restype = ctypes.c_double
     lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_quantize_row_e4m3.restype = None
+    lib.oracle_quantize_row_e4m3.argtypes = [c_p, c_p, c_p]
+    lib.oracle_append_kv.restype = ctypes.c_int
+    lib.oracle_append_kv.argtypes = [ctypes.c_int, ctypes.c_int, c_p, c_p, c_p, ctypes.c_int, c_p, ctypes.c_int,
+                                     c_p, ctypes.c_int, ctypes.c_int, c_p]
     return lib
 
 
@@ -152,3 +159,39 @@ def e4m3_to_f64(byte: int, lib=None) -> float:
 
 def bf16_to_f64(bits: int, lib=None) -> float:
     return (lib or load()).oracle_bf16_to_f64(bits)
+
+
+def e4m3_encode(x: float, lib=None) -> int:
+    """e4m3fn code of binary32 x (round to nearest even, clamped to +-448)."""
+    return int((lib or load()).oracle_e4m3_encode(float(x)))
+
+
+def quantize_row_e4m3(row_bf16, lib=None):
+    """One 576-value bf16 row -> (576 e4m3 codes as uint8, fp32 scale)."""
+    lib = lib or load()
+    r = _np(row_bf16, np.uint16).reshape(-1)
+    if r.shape[0] != 576:
+        raise ValueError("a cached row has 576 values")
+    codes = np.zeros((576,), dtype=np.uint8)
+    scale = np.zeros((1,), dtype=np.float32)
+    lib.oracle_quantize_row_e4m3(_ptr(r), _ptr(codes), _ptr(scale))
+    return codes, float(scale[0])
+
+
+def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, kv_dtype, lib=None):
+    """Oracle cache append: writes token t of sequence b at position
+    ctx_lens[b] - T + t of copies of the pages (and scales).  Returns
+    (pages, scales or None, ok) as numpy arrays; ok is False when a context or
+    page index was out of range (those tokens are skipped)."""
+    lib = lib or load()
+    kvd = KV_BF16 if kv_dtype in ("bf16", KV_BF16) else KV_FP8
+    ck = _np(c_kv_new, np.uint16)
+    kp = _np(k_pe_new, np.uint16)
+    B, T = int(ck.shape[0]), int(ck.shape[1])
+    pages = _np(kv_pages, np.uint16 if kvd == KV_BF16 else np.uint8).copy()
+    scales = _np(kv_scale, np.float32).copy() if kvd == KV_FP8 else None
+    pt = _np(page_table, np.int32)
+    cl = _np(ctx_lens, np.int32)
+    rc = lib.oracle_append_kv(B, T, _ptr(ck), _ptr(kp), _ptr(pages), kvd, _ptr(scales), int(pages.shape[0]),
+                              _ptr(pt), int(pt.shape[1]), int(pt.shape[1]), _ptr(cl))
+    return pages, scales, rc == 0

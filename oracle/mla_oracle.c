@@ -71,6 +71,92 @@ double oracle_e4m3_to_f64(uint8_t byte) {
     return sign ? -v : v;
 }
 
+/* FP8 e4m3fn encoding of a binary32 value, written from the same format
+ * definition: round to nearest, ties to even, magnitudes above 448 clamped to
+ * 448 (the cache writer clamps before it rounds), the sign kept (-0 -> 0x80).
+ * Subnormal codes m = 0..7 step 2^-9; a subnormal that rounds up to 8 steps
+ * is the smallest normal, whose code is also 8. */
+uint8_t oracle_e4m3_encode(float q) {
+    uint8_t sign = signbit(q) ? 0x80 : 0x00;
+    double a = fabs((double)q);
+    if (a > 448.0) a = 448.0;
+    if (a < ldexp(1.0, -6)) {                   /* subnormal range, quantum 2^-9 */
+        double n = a / ldexp(1.0, -9);          /* exact: a power-of-two scaling */
+        double r = nearbyint(n);                /* default rounding: ties to even */
+        return (uint8_t)(sign | (uint8_t)r);
+    }
+    int k;
+    frexp(a, &k);                               /* a = f 2^k, f in [0.5, 1) */
+    int e = k - 1;                              /* a in [2^e, 2^(e+1)) */
+    double n = a / ldexp(1.0, e - 3);           /* in [8, 16), exact */
+    double r = nearbyint(n);
+    if (r == 16.0) {
+        e += 1;
+        r = 8.0;
+    }
+    return (uint8_t)(sign | (uint8_t)(((e + 7) << 3) | ((int)r - 8)));
+}
+
+/* The cache writer for one token of an FP8 cache ("Kimi K2.6 DFlash on 8x
+ * MI300X", comparison of FP8 and BF16 KV: the FP8 cache computes a dynamic
+ * scale as it is written; here one fp32 scale per token):
+ *   x_d = widen(bf16 value d), d < 576       (c_kv 0..511 then k_pe)
+ *   scale = max_d |x_d| / 448 in binary32, or 1 when that is 0
+ *   code_d = e4m3(clamp(x_d / scale, -448, 448)), the division in binary32. */
+void oracle_quantize_row_e4m3(const uint16_t *row, uint8_t *codes, float *scale_out) {
+    float x[ORACLE_D];
+    float amax = 0.0f;
+    for (int d = 0; d < ORACLE_D; ++d) {
+        x[d] = (float)oracle_bf16_to_f64(row[d]);
+        float ax = fabsf(x[d]);
+        if (ax > amax) amax = ax;
+    }
+    float scale = amax / 448.0f;
+    if (!(scale > 0.0f)) scale = 1.0f;
+    for (int d = 0; d < ORACLE_D; ++d) {
+        float q = x[d] / scale;
+        if (q > 448.0f) q = 448.0f;
+        if (q < -448.0f) q = -448.0f;
+        codes[d] = oracle_e4m3_encode(q);
+    }
+    *scale_out = scale;
+}
+
+/* Append: token t of sequence b (its c_kv and k_pe, bf16) is cached position
+ * ctx_lens[b] - T + t, i.e. the context already counts the new tokens, as in
+ * the decode.  Returns 0, or -1 if a context or page index is out of range
+ * (nothing is written for such a token). */
+int oracle_append_kv(int B, int T, const uint16_t *c_kv_new, const uint16_t *k_pe_new, void *kv_pages, int kv_dtype,
+                     float *kv_scale, int num_pages, const int32_t *page_table, int page_table_stride,
+                     int max_pages, const int32_t *ctx_lens) {
+    int rc = 0;
+    for (int b = 0; b < B; ++b) {
+        int ctx = ctx_lens[b];
+        if (ctx < T || ctx > max_pages * ORACLE_PAGE) {
+            rc = -1;
+            continue;
+        }
+        for (int t = 0; t < T; ++t) {
+            int pos = ctx - T + t;
+            int page = page_table[(int64_t)b * page_table_stride + pos / ORACLE_PAGE];
+            if (page < 0 || page >= num_pages) {
+                rc = -1;
+                continue;
+            }
+            int64_t slot = (int64_t)page * ORACLE_PAGE + pos % ORACLE_PAGE;
+            uint16_t row[ORACLE_D];
+            memcpy(row, c_kv_new + ((int64_t)b * T + t) * ORACLE_DL, ORACLE_DL * sizeof(uint16_t));
+            memcpy(row + ORACLE_DL, k_pe_new + ((int64_t)b * T + t) * ORACLE_DR, ORACLE_DR * sizeof(uint16_t));
+            if (kv_dtype == ORACLE_KV_BF16) {
+                memcpy((uint16_t *)kv_pages + slot * ORACLE_D, row, sizeof row);
+            } else {
+                oracle_quantize_row_e4m3(row, (uint8_t *)kv_pages + slot * ORACLE_D, &kv_scale[slot]);
+            }
+        }
+    }
+    return rc;
+}
+
 typedef struct {
     int B, T, H;
     const uint16_t *q_lat;   /* [B,T,H,512] bf16 bits */

@@ -237,6 +237,83 @@ def pin_merge_rules(lib):
     assert np.allclose(mo, o2.mean(0), rtol=1e-14) and np.allclose(ml, math.log(2.0), rtol=1e-15)
 
 
+def pin_e4m3_encode_inverts_decoder(lib):
+    """The cache writer's encoder is the inverse of the (pinned) decoder on
+    every finite code, both zeros included."""
+    bad = [c for c in range(256)
+           if c not in (0x7F, 0xFF) and oracle.e4m3_encode(oracle.e4m3_to_f64(c, lib=lib), lib=lib) != c]
+    assert bad == [], bad[:8]
+
+
+def pin_e4m3_encode_rounding(lib):
+    """Round to nearest even with the clamp at 448, against torch's
+    float8_e4m3fn conversion: a dense grid past the clamp, every midpoint
+    between neighbouring codes (the ties) and the subnormal range."""
+    vals = [float(v) for v in torch.linspace(-480, 480, 9601, dtype=torch.float32)]
+    pos = sorted(oracle.e4m3_to_f64(c, lib=lib) for c in range(0x00, 0x7F))
+    mids = [(a + b) / 2 for a, b in zip(pos, pos[1:])]
+    vals += mids + [-m for m in mids] + [k * 2.0 ** -11 for k in range(-40, 41)]
+    x = torch.tensor(vals, dtype=torch.float32)
+    ref = x.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([oracle.e4m3_encode(float(v), lib=lib) for v in x.numpy()], dtype=np.uint8)
+    assert np.array_equal(ref, mine)
+
+
+def pin_row_quantiser(lib):
+    """Per-token quantiser = mla_workloads.quantize_fp8_rows (torch binary32
+    arithmetic: amax / 448, x / scale, clamp, round) bit for bit."""
+    gen = torch.Generator().manual_seed(11)
+    rows = (torch.randn((32, 576), generator=gen) * torch.rand((32, 1), generator=gen) * 8).to(torch.bfloat16)
+    rows[3] = 0
+    rows[4, 7] = -0.0
+    codes_ref, scales_ref = W.quantize_fp8_rows(rows.float())
+    for i in range(rows.shape[0]):
+        codes, scale = oracle.quantize_row_e4m3(rows[i], lib=lib)
+        assert np.array_equal(codes, codes_ref[i].numpy()), i
+        assert np.float32(scale) == scales_ref[i].numpy(), i
+
+
+def pin_append_positions(lib):
+    """Token t of sequence b lands at position ctx - T + t through the page
+    table, latent then RoPE values, and nothing else changes (bf16 cache:
+    exact copy of the written row)."""
+    gen = torch.Generator().manual_seed(12)
+    B, T, ctx = 3, 3, [5, 17, 40]
+    pages0, _, pt = W.build_paged_cache(ctx, W.KV_BF16, gen, shuffle=True)
+    c_new = torch.randn((B, T, 512), generator=gen).to(torch.bfloat16)
+    k_new = torch.randn((B, T, 64), generator=gen).to(torch.bfloat16)
+    pages, _, ok = oracle.append_kv(c_new, k_new, pages0, None, pt, torch.tensor(ctx, dtype=torch.int32),
+                                    kv_dtype=W.KV_BF16, lib=lib)
+    assert ok
+    expect = pages0.view(torch.int16).numpy().view(np.uint16).copy()
+    for b in range(B):
+        for t in range(T):
+            pos = ctx[b] - T + t
+            row = torch.cat([c_new[b, t], k_new[b, t]]).view(torch.int16).numpy().view(np.uint16)
+            expect[int(pt[b, pos // 16]), pos % 16] = row
+    assert np.array_equal(pages, expect)
+    # FP8 cache: the written rows are the generator's quantisation of the new rows
+    pages0, scales0, pt = W.build_paged_cache(ctx, W.KV_FP8, gen, shuffle=True)
+    pages, scales, ok = oracle.append_kv(c_new, k_new, pages0, scales0, pt, torch.tensor(ctx, dtype=torch.int32),
+                                         kv_dtype=W.KV_FP8, lib=lib)
+    assert ok
+    expect = pages0.numpy().copy()
+    expect_s = scales0.numpy().copy()
+    rows = torch.cat([c_new, k_new], dim=-1).float().reshape(B * T, 576)
+    codes, sc = W.quantize_fp8_rows(rows)
+    for b in range(B):
+        for t in range(T):
+            pos = ctx[b] - T + t
+            page, slot = int(pt[b, pos // 16]), pos % 16
+            expect[page, slot] = codes[b * T + t].numpy()
+            expect_s[page, slot] = sc[b * T + t].numpy()
+    assert np.array_equal(pages, expect)
+    assert np.array_equal(scales.view(np.uint32), expect_s.view(np.uint32)) or \
+        np.array_equal(np.isnan(scales), np.isnan(expect_s)) and np.array_equal(scales[~np.isnan(scales)],
+                                                                                expect_s[~np.isnan(expect_s)])
+
+
 PINS = [pin_e4m3_table, pin_bf16_widening, pin_library_attention, pin_single_position,
         pin_zero_query, pin_constant_values, pin_two_positions, pin_page_permutation,
-        pin_head_padding, pin_split_merge, pin_argmax_recovery, pin_merge_rules]
+        pin_head_padding, pin_split_merge, pin_argmax_recovery, pin_merge_rules,
+        pin_e4m3_encode_inverts_decoder, pin_e4m3_encode_rounding, pin_row_quantiser, pin_append_positions]

@@ -39,6 +39,12 @@ MUTANTS = {
     "head_token_swapped": ("int h = (int)(row % p->H);\n    int t = (int)((row / p->H) % p->T);",
                            "int t = (int)(row % p->T);\n    int h = (int)((row / p->T) % p->H);"),
     "weights_not_normalised": ("double w = exp(scores[j] - M) / Z;", "double w = exp(scores[j] - M);"),
+    "e4m3_encode_truncates": ("double r = nearbyint(n);                /* default rounding: ties to even */",
+                              "double r = floor(n);"),
+    "e4m3_encode_no_clamp": ("if (a > 448.0) a = 448.0;", ""),
+    "quantise_scale_447": ("float scale = amax / 448.0f;", "float scale = amax / 447.0f;"),
+    "append_position_shifted": ("int pos = ctx - T + t;", "int pos = ctx - T + t + 1;"),
+    "append_drops_rope": ("memcpy(row + ORACLE_DL, k_pe_new", "memset(row + ORACLE_DL, 0, 1); (void)(k_pe_new"),
 }
 
 
