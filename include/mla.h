@@ -200,6 +200,39 @@ MLA_API int mla_merge_partials(const float *out_parts, const float *lse_parts, i
                        mla_stream_t stream);
 
 /*
+ * Writes the T new tokens of every sequence into the paged cache: the step
+ * before mla_decode.  For an FP8 cache each token is quantised as it is
+ * written, with one fp32 scale per token ("Kimi K2.6 DFlash on 8x MI300X",
+ * comparison of FP8 and BF16 KV: the FP8 cache computes a dynamic scale):
+ *
+ *   x         = the token's 576 values, c_kv (512) then k_pe (64), widened
+ *   scale     = max|x| / 448 in binary32 (1 if that is 0)
+ *   code_d    = e4m3fn(clamp(x_d / scale, -448, 448)), round to nearest even
+ *
+ * A bf16 cache receives the values unchanged (kv_scale must be NULL).
+ *
+ *   c_kv_new   [B,T,512] bf16   16-byte aligned
+ *   k_pe_new   [B,T,64]  bf16   16-byte aligned
+ *   kv_pages   [P,16,576]       the cache (dims->kv_dtype), 16-byte aligned
+ *   kv_scale   [P,16] fp32      FP8 only
+ *   page_table, ctx_lens        as for mla_decode; ctx_lens[b] already counts
+ *                               the T new tokens, so token t of sequence b
+ *                               goes to position ctx_lens[b] - T + t
+ *   dims                        B, T (1..8), num_pages, max_pages_per_seq,
+ *                               page_table_stride, kv_dtype are read
+ *   device_error               NULL, or a device {code, info} pair that
+ *                               receives MLA_DEV_BAD_CTX (ctx < T or beyond the
+ *                               page table) or MLA_DEV_BAD_PAGE like the
+ *                               workspace error word; such tokens are skipped
+ *
+ * Inputs must be finite.  Asynchronous on `stream`; writes only the new
+ * tokens' slots (and their scales).
+ */
+MLA_API int mla_append_kv(const void *c_kv_new, const void *k_pe_new, void *kv_pages, float *kv_scale,
+                          const int32_t *page_table, const int32_t *ctx_lens, const mla_dims *dims,
+                          int32_t *device_error, mla_stream_t stream);
+
+/*
  * Copies the workspace error word to the host.  SYNCHRONISES `stream`.
  * *code receives an mla_device_error (the first one raised since the last
  * reset), *info its detail (may be NULL).

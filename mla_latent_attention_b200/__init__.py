@@ -16,7 +16,7 @@ import threading
 
 import torch
 
-__all__ = ["decode", "merge_partials", "workspace_size", "read_device_error",
+__all__ = ["decode", "merge_partials", "append_kv", "workspace_size", "read_device_error",
            "reset_device_error", "library_path", "load_library", "MlaError", "KERNELS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +29,7 @@ KV_BF16, KV_FP8 = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 KERNELS = {"auto": 0, "simt": 1, "tcgen05": 2}
 DEV_ERRORS = {0: "ok", 1: "bad page index", 2: "bad context length", 3: "bad visible count"}
-EXPORTED = ("mla_decode_workspace_size", "mla_decode", "mla_decode_noalloc", "mla_merge_partials",
+EXPORTED = ("mla_decode_workspace_size", "mla_decode", "mla_decode_noalloc", "mla_merge_partials", "mla_append_kv",
             "mla_read_device_error", "mla_reset_device_error", "mla_status_string",
             "mla_last_cuda_error")
 
@@ -73,6 +73,8 @@ def load_library(path: str = None):
                                            ctypes.POINTER(Dims), vp]
         lib.mla_merge_partials.restype = ctypes.c_int
         lib.mla_merge_partials.argtypes = [vp, vp, i32, i64, vp, i32, vp, vp]
+        lib.mla_append_kv.restype = ctypes.c_int
+        lib.mla_append_kv.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(Dims), vp, vp]
         lib.mla_read_device_error.restype = ctypes.c_int
         lib.mla_read_device_error.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), vp]
         lib.mla_reset_device_error.restype = ctypes.c_int
@@ -224,6 +226,32 @@ def merge_partials(out_parts, lse_parts, *, out=None, lse=None, out_dtype=torch.
                                 _stream(stream, dev))
     _check(rc, "mla_merge_partials")
     return out, lse
+
+
+def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, device_error=None,
+              stream=None):
+    """Write the T new tokens of each sequence into the paged cache
+    (``mla_append_kv``): token t of sequence b goes to position
+    ctx_lens[b] - T + t.  c_kv_new [B,T,512] and k_pe_new [B,T,64] are bf16;
+    an FP8 cache is quantised with one scale per token.  ``device_error``: an
+    optional int32 CUDA tensor of 2 elements receiving a device error."""
+    lib = load_library()
+    dev = kv_pages.device
+    B, T = int(c_kv_new.shape[0]), int(c_kv_new.shape[1])
+    _need(c_kv_new, "c_kv_new", torch.bfloat16, dev, (B, T, 512))
+    _need(k_pe_new, "k_pe_new", torch.bfloat16, dev, (B, T, 64))
+    _need(page_table, "page_table", torch.int32, dev)
+    _need(ctx_lens, "ctx_lens", torch.int32, dev, (B,))
+    if kv_scale is not None:
+        _need(kv_scale, "kv_scale", torch.float32, dev)
+    if device_error is not None:
+        _need(device_error, "device_error", torch.int32, dev, (2,))
+    dims = Dims(B=B, T=T, H=1, num_pages=int(kv_pages.shape[0]), max_pages_per_seq=int(page_table.shape[1]),
+                page_table_stride=int(page_table.stride(0)), kv_dtype=_kv_code(kv_pages), out_dtype=OUT_BF16,
+                num_splits=0, kernel=0, vis_lens=None, stage_event=None)
+    rc = lib.mla_append_kv(_ptr(c_kv_new), _ptr(k_pe_new), _ptr(kv_pages), _ptr(kv_scale), _ptr(page_table),
+                           _ptr(ctx_lens), ctypes.byref(dims), _ptr(device_error), _stream(stream, dev))
+    _check(rc, "mla_append_kv")
 
 
 def read_device_error(workspace, stream=None):

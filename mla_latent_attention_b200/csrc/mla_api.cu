@@ -247,6 +247,25 @@ int mla_merge_partials(const float *out_parts, const float *lse_parts, int32_t n
                                lse_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int mla_append_kv(const void *c_kv_new, const void *k_pe_new, void *kv_pages, float *kv_scale,
+                  const int32_t *page_table, const int32_t *ctx_lens, const mla_dims *d, int32_t *device_error,
+                  mla_stream_t stream) {
+    if (!c_kv_new || !k_pe_new || !kv_pages || !page_table || !ctx_lens || !d) return MLA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->T < 1 || d->T > kMaxT || d->num_pages < 1 || d->max_pages_per_seq < 1 ||
+        d->page_table_stride < d->max_pages_per_seq)
+        return MLA_ERR_INVALID_ARG;
+    if ((int64_t)d->B * d->T > (int64_t)INT32_MAX) return MLA_ERR_INVALID_ARG;
+    const bool fp8 = d->kv_dtype == MLA_KV_FP8_E4M3;
+    if (!fp8 && d->kv_dtype != MLA_KV_BF16) return MLA_ERR_INVALID_ARG;
+    if (fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
+    if (!aligned(c_kv_new, 16) || !aligned(k_pe_new, 16) || !aligned(kv_pages, 16) || !aligned(page_table, 4) ||
+        !aligned(ctx_lens, 4) || (kv_scale && !aligned(kv_scale, 4)) || (device_error && !aligned(device_error, 4)))
+        return MLA_ERR_INVALID_ARG;
+    return launch_append(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, d->B, d->T, d->num_pages,
+                         d->max_pages_per_seq, d->page_table_stride, fp8, device_error,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
 int mla_read_device_error(const void *workspace, int32_t *code, int32_t *info, mla_stream_t stream) {
     if (!workspace || !code) return MLA_ERR_INVALID_ARG;
     int32_t word[2] = {0, 0};

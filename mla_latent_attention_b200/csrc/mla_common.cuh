@@ -241,6 +241,9 @@ __device__ __forceinline__ void store_out(void *out, int64_t idx, float v, int o
 
 // Host-side launch helpers implemented per kernel family.
 int launch_simt(const Problem &p, cudaStream_t stream);
+int launch_append(const void *c_kv_new, const void *k_pe_new, void *kv_pages, float *kv_scale,
+                  const int32_t *page_table, const int32_t *ctx_lens, int B, int T, int num_pages, int max_pages,
+                  int pt_stride, int fp8, int32_t *err, cudaStream_t stream);
 int launch_tc(const Problem &p, cudaStream_t stream);
 int launch_merge_internal(const Problem &p, cudaStream_t stream);
 int launch_merge_public(const float *out_parts, const float *lse_parts, int n_parts, int64_t rows,

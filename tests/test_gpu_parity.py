@@ -38,6 +38,9 @@ SMALL = [
     ("long_ctx_142k", dict(ctx_override=("fixed", 9001))),
     ("long_ctx_142k", dict(ctx_override=("fixed", 5003), kv=W.KV_BF16)),
     ("ragged_dcp8", dict(B=5, ctx_override=("loguniform", 40, 3000))),
+    # deeper drafts: T = 1 + st for st = 4 and 7
+    ("spec_verify_small", dict(B=3, T=5, ctx_override=("uniform", 300, 1500))),
+    ("batched_verify_fp8_32k", dict(B=2, T=8, ctx_override=("fixed", 900))),
 ]
 
 
