@@ -1,0 +1,72 @@
+"""Context-parallel decode over CPU ranks (gloo): each rank decodes its
+round-robin share of the positions, the partials are all-gathered and merged.
+The per-rank decode and the merge are stand-ins built on the oracle (this is a
+test of the exchange and of the partitioning, not of the kernels); the merged
+answer must equal the oracle's decode of the whole cache."""
+import datetime
+import multiprocessing as mp
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, kv, queue):
+    import mla_workloads as W
+    import oracle
+    from mla_latent_attention_b200 import dcp
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = W.make_workload("ragged_dcp8", B=3, H=4, kv=kv, ctx_override=("loguniform", 30, 400))
+        part = W.partition_round_robin(w, world)[rank]
+        B, T, H = w.B, w.T, w.H
+
+        def decode_fn(q_lat, q_pe, pages, scale, pt, cl, sm, vis):
+            o, l = oracle.decode(q_lat, q_pe, pages, scale, pt, cl, sm, kv_dtype=kv, vis_lens=vis)
+            return (torch.from_numpy(o).to(torch.float32).view(B, T, H, 512),
+                    torch.from_numpy(l).to(torch.float32).view(B, T, H))
+
+        def merge_fn(o_all, l_all, out_dtype):
+            n = o_all.shape[0]
+            mo, ml = oracle.merge(o_all.double().reshape(n, -1, 512).numpy(), l_all.double().reshape(n, -1).numpy())
+            return torch.from_numpy(mo).view(B, T, H, 512), torch.from_numpy(ml).view(B, T, H)
+
+        out, lse = dcp.dcp_decode(part.q_lat, part.q_pe, part.kv_pages, part.kv_scale, part.page_table,
+                                  part.ctx_lens, part.sm_scale, vis_lens=part.vis_lens, decode_fn=decode_fn,
+                                  merge_fn=merge_fn)
+        ref_o, ref_l = oracle.decode_workload(w)
+        err_o = float(np.abs(out.reshape(-1, 512).numpy() - ref_o).max())
+        err_l = float(np.abs(lse.reshape(-1).numpy() - ref_l).max())
+        queue.put((rank, err_o, err_l, float(np.abs(ref_o).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
+def test_dcp_over_cpu_ranks_equals_whole_decode(world, kv):
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, kv, queue)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [queue.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err_o, err_l, scale in results:
+        # fp32 partials, exact merge: rounding only
+        assert err_o <= 1e-6 * scale + 1e-7, (rank, err_o)
+        assert err_l <= 1e-5, (rank, err_l)
