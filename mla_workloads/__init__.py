@@ -320,6 +320,20 @@ def partition_round_robin(w: Workload, n_parts: int, gen_seed: int = 77) -> list
     return parts
 
 
+def static_scale_workload(w: Workload) -> Workload:
+    """The same FP8 workload re-quantised with one per-tensor scale: the
+    dequantised cache values (unused slots stay NaN) divided by
+    s = max|value| / 448, rounded to e4m3; kv_scale becomes the one-element
+    tensor [s]."""
+    if w.kv_dtype != KV_FP8:
+        raise ValueError("a static scale applies to FP8 caches")
+    v = w.kv_pages.view(torch.float8_e4m3fn).to(torch.float32) * w.kv_scale.unsqueeze(-1)
+    s = torch.nan_to_num(v.abs(), nan=0.0).amax() / FP8_MAX
+    s = torch.where(s > 0, s, torch.ones_like(s)).to(torch.float32)
+    codes = (v / s).clamp(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+    return dataclasses.replace(w, kv_pages=codes, kv_scale=s.reshape(1))
+
+
 def permute_pages(w: Workload, seed: int = 5) -> Workload:
     """Same logical cache with physical pages relabelled by a random permutation."""
     gen = torch.Generator(device="cpu")

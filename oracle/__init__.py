@@ -57,7 +57,7 @@ def _bind(lib):
     c_p = ctypes.c_void_p
     lib.oracle_mla_decode.restype = ctypes.c_int
     lib.oracle_mla_decode.argtypes = [
-        ctypes.c_int, ctypes.c_int, ctypes.c_int, c_p, c_p, c_p, ctypes.c_int, c_p, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, c_p, c_p, c_p, ctypes.c_int, c_p, ctypes.c_int, ctypes.c_int,
         c_p, ctypes.c_int, c_p, c_p, ctypes.c_double, c_p, ctypes.c_int64, c_p, c_p, ctypes.c_int]
     lib.oracle_mla_merge.restype = ctypes.c_int
     lib.oracle_mla_merge.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, c_p, c_p, c_p, c_p]
@@ -68,10 +68,10 @@ def _bind(lib):
     lib.oracle_e4m3_encode.restype = ctypes.c_uint8
     lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
     lib.oracle_quantize_row_e4m3.restype = None
-    lib.oracle_quantize_row_e4m3.argtypes = [c_p, c_p, c_p]
+    lib.oracle_quantize_row_e4m3.argtypes = [c_p, c_p, c_p, ctypes.c_float]
     lib.oracle_append_kv.restype = ctypes.c_int
     lib.oracle_append_kv.argtypes = [ctypes.c_int, ctypes.c_int, c_p, c_p, c_p, ctypes.c_int, c_p, ctypes.c_int,
-                                     c_p, ctypes.c_int, ctypes.c_int, c_p]
+                                     ctypes.c_int, c_p, ctypes.c_int, ctypes.c_int, c_p]
     return lib
 
 
@@ -109,7 +109,8 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, k
 
     q_lat [B,T,H,512] and q_pe [B,T,H,64] are bf16 (torch bf16 tensors or uint16
     bit arrays); kv_pages [P,16,576] is bf16 or e4m3fn bytes; kv_scale [P,16]
-    fp32 for FP8.  ``rows`` lists flat row ids b*T*H + t*H + h (default: all).
+    fp32 for FP8, or a single value (a per-tensor static scale).  ``rows``
+    lists flat row ids b*T*H + t*H + h (default: all).
     """
     lib = lib or load()
     B, T, H = int(q_lat.shape[0]), int(q_lat.shape[1]), int(q_lat.shape[2])
@@ -118,6 +119,7 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, k
     qp = _np(q_pe, np.uint16)
     kv = _np(kv_pages, np.uint16 if kvd == KV_BF16 else np.uint8)
     sc = _np(kv_scale, np.float32) if kvd == KV_FP8 else None
+    per_tensor = int(sc is not None and sc.size == 1)
     pt = _np(page_table, np.int32)
     cl = _np(ctx_lens, np.int32)
     vl = _np(vis_lens, np.int32)
@@ -125,7 +127,7 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, k
     n_rows = B * T * H if rr is None else int(rr.shape[0])
     out = np.zeros((n_rows, 512), dtype=np.float64)
     lse = np.zeros((n_rows,), dtype=np.float64)
-    rc = lib.oracle_mla_decode(B, T, H, _ptr(ql), _ptr(qp), _ptr(kv), kvd, _ptr(sc),
+    rc = lib.oracle_mla_decode(B, T, H, _ptr(ql), _ptr(qp), _ptr(kv), kvd, _ptr(sc), per_tensor,
                                int(kv.shape[0]), _ptr(pt), int(pt.shape[1]), _ptr(cl), _ptr(vl),
                                float(sm_scale), _ptr(rr), n_rows, _ptr(out), _ptr(lse), int(threads))
     if rc != 0:
@@ -174,7 +176,7 @@ def quantize_row_e4m3(row_bf16, lib=None):
         raise ValueError("a cached row has 576 values")
     codes = np.zeros((576,), dtype=np.uint8)
     scale = np.zeros((1,), dtype=np.float32)
-    lib.oracle_quantize_row_e4m3(_ptr(r), _ptr(codes), _ptr(scale))
+    lib.oracle_quantize_row_e4m3(_ptr(r), _ptr(codes), _ptr(scale), ctypes.c_float(0.0))
     return codes, float(scale[0])
 
 
@@ -190,8 +192,10 @@ def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, k
     B, T = int(ck.shape[0]), int(ck.shape[1])
     pages = _np(kv_pages, np.uint16 if kvd == KV_BF16 else np.uint8).copy()
     scales = _np(kv_scale, np.float32).copy() if kvd == KV_FP8 else None
+    per_tensor = int(scales is not None and scales.size == 1)
     pt = _np(page_table, np.int32)
     cl = _np(ctx_lens, np.int32)
-    rc = lib.oracle_append_kv(B, T, _ptr(ck), _ptr(kp), _ptr(pages), kvd, _ptr(scales), int(pages.shape[0]),
+    rc = lib.oracle_append_kv(B, T, _ptr(ck), _ptr(kp), _ptr(pages), kvd, _ptr(scales), per_tensor,
+                              int(pages.shape[0]),
                               _ptr(pt), int(pt.shape[1]), int(pt.shape[1]), _ptr(cl))
     return pages, scales, rc == 0

@@ -103,7 +103,9 @@ uint8_t oracle_e4m3_encode(float q) {
  *   x_d = widen(bf16 value d), d < 576       (c_kv 0..511 then k_pe)
  *   scale = max_d |x_d| / 448 in binary32, or 1 when that is 0
  *   code_d = e4m3(clamp(x_d / scale, -448, 448)), the division in binary32. */
-void oracle_quantize_row_e4m3(const uint16_t *row, uint8_t *codes, float *scale_out) {
+/* static_scale > 0: a per-tensor scale given by the caller replaces the
+ * row's own (a static, calibrated scale). */
+void oracle_quantize_row_e4m3(const uint16_t *row, uint8_t *codes, float *scale_out, float static_scale) {
     float x[ORACLE_D];
     float amax = 0.0f;
     for (int d = 0; d < ORACLE_D; ++d) {
@@ -113,6 +115,7 @@ void oracle_quantize_row_e4m3(const uint16_t *row, uint8_t *codes, float *scale_
     }
     float scale = amax / 448.0f;
     if (!(scale > 0.0f)) scale = 1.0f;
+    if (static_scale > 0.0f) scale = static_scale;
     for (int d = 0; d < ORACLE_D; ++d) {
         float q = x[d] / scale;
         if (q > 448.0f) q = 448.0f;
@@ -127,8 +130,8 @@ void oracle_quantize_row_e4m3(const uint16_t *row, uint8_t *codes, float *scale_
  * the decode.  Returns 0, or -1 if a context or page index is out of range
  * (nothing is written for such a token). */
 int oracle_append_kv(int B, int T, const uint16_t *c_kv_new, const uint16_t *k_pe_new, void *kv_pages, int kv_dtype,
-                     float *kv_scale, int num_pages, const int32_t *page_table, int page_table_stride,
-                     int max_pages, const int32_t *ctx_lens) {
+                     float *kv_scale, int kv_scale_per_tensor, int num_pages, const int32_t *page_table,
+                     int page_table_stride, int max_pages, const int32_t *ctx_lens) {
     int rc = 0;
     for (int b = 0; b < B; ++b) {
         int ctx = ctx_lens[b];
@@ -150,7 +153,10 @@ int oracle_append_kv(int B, int T, const uint16_t *c_kv_new, const uint16_t *k_p
             if (kv_dtype == ORACLE_KV_BF16) {
                 memcpy((uint16_t *)kv_pages + slot * ORACLE_D, row, sizeof row);
             } else {
-                oracle_quantize_row_e4m3(row, (uint8_t *)kv_pages + slot * ORACLE_D, &kv_scale[slot]);
+                float s;
+                oracle_quantize_row_e4m3(row, (uint8_t *)kv_pages + slot * ORACLE_D, &s,
+                                         kv_scale_per_tensor ? kv_scale[0] : 0.0f);
+                if (!kv_scale_per_tensor) kv_scale[slot] = s;
             }
         }
     }
@@ -163,7 +169,8 @@ typedef struct {
     const uint16_t *q_pe;    /* [B,T,H,64]  bf16 bits */
     const void *kv_pages;    /* [P,16,576] bf16 bits or e4m3fn bytes */
     int kv_dtype;
-    const float *kv_scale;   /* [P,16] for FP8, else NULL */
+    const float *kv_scale;   /* [P,16] for FP8, or [1] with kv_scale_per_tensor; else NULL */
+    int kv_scale_per_tensor;
     int num_pages;
     const int32_t *page_table;
     int page_table_stride;
@@ -180,7 +187,7 @@ static double kv_value(const oracle_problem *p, int64_t page, int slot, int d) {
         return oracle_bf16_to_f64(kv[row * ORACLE_D + d]);
     } else {
         const uint8_t *kv = (const uint8_t *)p->kv_pages;
-        return oracle_e4m3_to_f64(kv[row * ORACLE_D + d]) * (double)p->kv_scale[row];
+        return oracle_e4m3_to_f64(kv[row * ORACLE_D + d]) * (double)p->kv_scale[p->kv_scale_per_tensor ? 0 : row];
     }
 }
 
@@ -298,7 +305,8 @@ static int run_rows(const oracle_problem *p, const int64_t *rows, int64_t n_rows
 /* Decode every row (rows == NULL) or the listed flat rows b*T*H + t*H + h.
  * out: [n_rows, 512] fp64, lse: [n_rows] fp64.  Returns 0 on success. */
 int oracle_mla_decode(int B, int T, int H, const uint16_t *q_lat, const uint16_t *q_pe,
-                      const void *kv_pages, int kv_dtype, const float *kv_scale, int num_pages,
+                      const void *kv_pages, int kv_dtype, const float *kv_scale, int kv_scale_per_tensor,
+                      int num_pages,
                       const int32_t *page_table, int page_table_stride, const int32_t *ctx_lens,
                       const int32_t *vis_lens, double sm_scale, const int64_t *rows,
                       int64_t n_rows, double *out, double *lse, int n_threads) {
@@ -311,6 +319,7 @@ int oracle_mla_decode(int B, int T, int H, const uint16_t *q_lat, const uint16_t
     p.kv_pages = kv_pages;
     p.kv_dtype = kv_dtype;
     p.kv_scale = kv_scale;
+    p.kv_scale_per_tensor = kv_scale_per_tensor;
     p.num_pages = num_pages;
     p.page_table = page_table;
     p.page_table_stride = page_table_stride;

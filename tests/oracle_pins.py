@@ -313,7 +313,36 @@ def pin_append_positions(lib):
                                                                                 expect_s[~np.isnan(expect_s)])
 
 
+def pin_static_scale(lib):
+    """A per-tensor scale s is the per-position cache whose every scale is s:
+    both decode to the same bits; and the writer with a static scale stores
+    e4m3(clamp(x / s)) (torch arithmetic) and leaves the scale alone."""
+    w = W.make_workload("spec_verify_small", B=2, kv=W.KV_FP8, ctx_override=("uniform", 40, 90))
+    ws = W.static_scale_workload(w)
+    s = float(ws.kv_scale[0])
+    full = ws.kv_scale.expand(ws.kv_pages.shape[0], 16).contiguous()
+    o1, l1 = oracle.decode(ws.q_lat, ws.q_pe, ws.kv_pages, ws.kv_scale, ws.page_table, ws.ctx_lens, ws.sm_scale,
+                           kv_dtype=W.KV_FP8, lib=lib)
+    o2, l2 = oracle.decode(ws.q_lat, ws.q_pe, ws.kv_pages, full, ws.page_table, ws.ctx_lens, ws.sm_scale,
+                           kv_dtype=W.KV_FP8, lib=lib)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    gen = torch.Generator().manual_seed(14)
+    c_new = (torch.randn((2, 3, 512), generator=gen) * 3).to(torch.bfloat16)
+    k_new = torch.randn((2, 3, 64), generator=gen).to(torch.bfloat16)
+    pages, scales, ok = oracle.append_kv(c_new, k_new, ws.kv_pages, ws.kv_scale, ws.page_table, ws.ctx_lens,
+                                         kv_dtype=W.KV_FP8, lib=lib)
+    assert ok and scales.shape == (1,) and np.float32(scales[0]) == np.float32(s)
+    rows = torch.cat([c_new, k_new], dim=-1).float()
+    codes = (rows / torch.tensor(s, dtype=torch.float32)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    ctx = ws.ctx_lens.tolist()
+    for b in range(2):
+        for t in range(3):
+            pos = ctx[b] - 3 + t
+            assert np.array_equal(pages[int(ws.page_table[b, pos // 16]), pos % 16], codes[b, t].numpy())
+
+
 PINS = [pin_e4m3_table, pin_bf16_widening, pin_library_attention, pin_single_position,
         pin_zero_query, pin_constant_values, pin_two_positions, pin_page_permutation,
         pin_head_padding, pin_split_merge, pin_argmax_recovery, pin_merge_rules,
-        pin_e4m3_encode_inverts_decoder, pin_e4m3_encode_rounding, pin_row_quantiser, pin_append_positions]
+        pin_e4m3_encode_inverts_decoder, pin_e4m3_encode_rounding, pin_row_quantiser, pin_append_positions,
+        pin_static_scale]

@@ -31,7 +31,7 @@ MUTANTS = {
     "e4m3_subnormal_exp": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
     "value_reads_shifted": ("out[d] += w * kv_value(p, page, slot, d);",
                             "out[d] += w * kv_value(p, page, slot, d + 1);"),
-    "fp8_scale_dropped": ("* (double)p->kv_scale[row];", "* 1.0;"),
+    "fp8_scale_dropped": ("* (double)p->kv_scale[p->kv_scale_per_tensor ? 0 : row];", "* 1.0;"),
     "lse_base2": ("*lse = M + log(Z);", "*lse = M + log2(Z);"),
     "sm_scale_dropped": ("scores[j] = p->sm_scale * dot;", "scores[j] = dot;"),
     "merge_unweighted": ("double w = exp(l - L);", "double w = 1.0;"),
