@@ -107,6 +107,10 @@ typedef struct mla_dims {
                                    attention kernel and before the merge kernel (inside a stream
                                    capture as an external event node, readable after each
                                    replay); NULL for none */
+    int32_t kv_scale_per_tensor;  /* FP8 only: 0 = kv_scale is [P,16], one scale per cached
+                                     position; 1 = kv_scale points to ONE fp32 scale for the
+                                     whole cache (a static, calibrated scale: "Kimi K2.6 DFlash
+                                     on 8x MI300X", next steps) */
 } mla_dims;
 
 /*
@@ -128,7 +132,8 @@ MLA_API int64_t mla_decode_workspace_size(const mla_dims *dims);
  *                                   512..575 are k_pe.  16-byte aligned.
  *   kv_scale   [P,16] fp32          FP8 only: dequantised value = e4m3 * scale
  *                                   of its position.  16-byte aligned.  Must be
- *                                   NULL for bf16.
+ *                                   NULL for bf16.  With dims->kv_scale_per_tensor
+ *                                   it is one fp32 scale for every position.
  *   page_table [B, stride] int32    page_table[b][i] = physical page of the
  *                                   sequence's positions 16i .. 16i+15.  Only
  *                                   entries i < ceil(ctx_lens[b]/16) are read.
@@ -214,7 +219,8 @@ MLA_API int mla_merge_partials(const float *out_parts, const float *lse_parts, i
  *   c_kv_new   [B,T,512] bf16   16-byte aligned
  *   k_pe_new   [B,T,64]  bf16   16-byte aligned
  *   kv_pages   [P,16,576]       the cache (dims->kv_dtype), 16-byte aligned
- *   kv_scale   [P,16] fp32      FP8 only
+ *   kv_scale   [P,16] fp32      FP8 only; with dims->kv_scale_per_tensor one
+ *                               fp32 static scale, read and left unchanged
  *   page_table, ctx_lens        as for mla_decode; ctx_lens[b] already counts
  *                               the T new tokens, so token t of sequence b
  *                               goes to position ctx_lens[b] - T + t

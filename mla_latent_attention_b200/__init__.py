@@ -44,7 +44,7 @@ class Dims(ctypes.Structure):
                 ("page_table_stride", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
                 ("out_dtype", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("kernel", ctypes.c_int32), ("vis_lens", ctypes.c_void_p),
-                ("stage_event", ctypes.c_void_p)]
+                ("stage_event", ctypes.c_void_p), ("kv_scale_per_tensor", ctypes.c_int32)]
 
 
 def library_path() -> str:
@@ -115,7 +115,7 @@ def _kv_code(kv_pages):
 
 
 def make_dims(q_lat, kv_pages, page_table, *, out_dtype=torch.bfloat16, num_splits=0,
-              kernel="auto", vis_lens=None, stage_event=None) -> Dims:
+              kernel="auto", vis_lens=None, stage_event=None, kv_scale=None) -> Dims:
     B, T, H = int(q_lat.shape[0]), int(q_lat.shape[1]), int(q_lat.shape[2])
     return Dims(B=B, T=T, H=H, num_pages=int(kv_pages.shape[0]),
                 max_pages_per_seq=int(page_table.shape[1]),
@@ -123,7 +123,8 @@ def make_dims(q_lat, kv_pages, page_table, *, out_dtype=torch.bfloat16, num_spli
                 out_dtype=OUT_F32 if out_dtype == torch.float32 else OUT_BF16,
                 num_splits=int(num_splits), kernel=KERNELS[kernel],
                 vis_lens=None if vis_lens is None else vis_lens.data_ptr(),
-                stage_event=None if stage_event is None else stage_event.cuda_event)
+                stage_event=None if stage_event is None else stage_event.cuda_event,
+                kv_scale_per_tensor=int(kv_scale is not None and kv_scale.numel() == 1))
 
 
 def workspace_size(dims: Dims) -> int:
@@ -161,8 +162,9 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, o
     _need(kv_pages, "kv_pages", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), dev)
     if kv_pages.dim() != 3 or kv_pages.shape[1:] != (16, 576):
         raise MlaError(f"kv_pages must be [P,16,576], got {tuple(kv_pages.shape)}")
-    if kv_scale is not None:
-        _need(kv_scale, "kv_scale", torch.float32, dev, (kv_pages.shape[0], 16))
+    if kv_scale is not None:  # per position [P,16], or one per-tensor static scale
+        _need(kv_scale, "kv_scale", torch.float32, dev,
+              (1,) if kv_scale.numel() == 1 else (kv_pages.shape[0], 16))
     _need(page_table, "page_table", torch.int32, dev)
     if page_table.dim() != 2 or page_table.shape[0] != B or page_table.stride(1) != 1:
         raise MlaError("page_table must be [B, max_pages] int32 with unit column stride")
@@ -179,7 +181,7 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, o
     else:
         _need(lse, "lse", torch.float32, dev, (B, T, H))
     dims = make_dims(q_lat, kv_pages, page_table, out_dtype=out_dtype, num_splits=num_splits,
-                     kernel=kernel, vis_lens=vis_lens, stage_event=stage_event)
+                     kernel=kernel, vis_lens=vis_lens, stage_event=stage_event, kv_scale=kv_scale)
     need = workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -233,7 +235,8 @@ def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, d
     """Write the T new tokens of each sequence into the paged cache
     (``mla_append_kv``): token t of sequence b goes to position
     ctx_lens[b] - T + t.  c_kv_new [B,T,512] and k_pe_new [B,T,64] are bf16;
-    an FP8 cache is quantised with one scale per token.  ``device_error``: an
+    an FP8 cache is quantised with one scale per token (written to kv_scale
+    [P,16]), or with the static scale when kv_scale has one element.  ``device_error``: an
     optional int32 CUDA tensor of 2 elements receiving a device error."""
     lib = load_library()
     dev = kv_pages.device
@@ -248,7 +251,8 @@ def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, d
         _need(device_error, "device_error", torch.int32, dev, (2,))
     dims = Dims(B=B, T=T, H=1, num_pages=int(kv_pages.shape[0]), max_pages_per_seq=int(page_table.shape[1]),
                 page_table_stride=int(page_table.stride(0)), kv_dtype=_kv_code(kv_pages), out_dtype=OUT_BF16,
-                num_splits=0, kernel=0, vis_lens=None, stage_event=None)
+                num_splits=0, kernel=0, vis_lens=None, stage_event=None,
+                kv_scale_per_tensor=int(kv_scale is not None and kv_scale.numel() == 1))
     rc = lib.mla_append_kv(_ptr(c_kv_new), _ptr(k_pe_new), _ptr(kv_pages), _ptr(kv_scale), _ptr(page_table),
                            _ptr(ctx_lens), ctypes.byref(dims), _ptr(device_error), _stream(stream, dev))
     _check(rc, "mla_append_kv")

@@ -49,6 +49,8 @@ int check_dims(const mla_dims *d) {
     if (d->num_pages < 1 || d->max_pages_per_seq < 1 || d->page_table_stride < d->max_pages_per_seq)
         return MLA_ERR_INVALID_ARG;
     if (d->kv_dtype != MLA_KV_BF16 && d->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+    if (d->kv_scale_per_tensor != 0 && d->kv_scale_per_tensor != 1) return MLA_ERR_INVALID_ARG;
+    if (d->kv_scale_per_tensor && d->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
     if (d->out_dtype != MLA_OUT_BF16 && d->out_dtype != MLA_OUT_F32) return MLA_ERR_INVALID_ARG;
     if (d->num_splits < 0) return MLA_ERR_INVALID_ARG;
     if (d->kernel != MLA_KERNEL_AUTO && d->kernel != MLA_KERNEL_SIMT && d->kernel != MLA_KERNEL_TCGEN05)
@@ -145,6 +147,7 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     p.max_pages = dims->max_pages_per_seq;
     p.pt_stride = dims->page_table_stride;
     p.out_f32 = dims->out_dtype == MLA_OUT_F32;
+    p.kv_scale_per_tensor = dims->kv_scale_per_tensor;
     p.n_slots = pl.n_slots;
     p.n_groups = pl.n_groups;
     p.rows_per_group = pl.rows_per_group;
@@ -257,12 +260,14 @@ int mla_append_kv(const void *c_kv_new, const void *k_pe_new, void *kv_pages, fl
     if ((int64_t)d->B * d->T > (int64_t)INT32_MAX) return MLA_ERR_INVALID_ARG;
     const bool fp8 = d->kv_dtype == MLA_KV_FP8_E4M3;
     if (!fp8 && d->kv_dtype != MLA_KV_BF16) return MLA_ERR_INVALID_ARG;
+    if (d->kv_scale_per_tensor != 0 && d->kv_scale_per_tensor != 1) return MLA_ERR_INVALID_ARG;
+    if (d->kv_scale_per_tensor && !fp8) return MLA_ERR_INVALID_ARG;
     if (fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
     if (!aligned(c_kv_new, 16) || !aligned(k_pe_new, 16) || !aligned(kv_pages, 16) || !aligned(page_table, 4) ||
         !aligned(ctx_lens, 4) || (kv_scale && !aligned(kv_scale, 4)) || (device_error && !aligned(device_error, 4)))
         return MLA_ERR_INVALID_ARG;
     return launch_append(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, d->B, d->T, d->num_pages,
-                         d->max_pages_per_seq, d->page_table_stride, fp8, device_error,
+                         d->max_pages_per_seq, d->page_table_stride, fp8, d->kv_scale_per_tensor, device_error,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -31,6 +31,7 @@ struct AppendArgs {
     const int32_t *ctx_lens;        // [B]
     int32_t *err;                   // {code, info} or null
     int B, T, num_pages, max_pages, pt_stride;
+    int per_tensor;                 // FP8: kv_scale[0] is the cache's static scale (read, not written)
 };
 
 __device__ __forceinline__ void append_error(int32_t *err, int code, int info) {
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendArgs a) {
         amax = fmaxf(fmaxf(wmax[0], wmax[1]), wmax[2]);
         float scale = __fdiv_rn(amax, 448.f);
         if (!(scale > 0.f)) scale = 1.f;
+        if (a.per_tensor) scale = __ldg(a.kv_scale);
         if (tid < kUnits) {
             uint32_t w[2];
 #pragma unroll
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendArgs a) {
             }
             reinterpret_cast<uint2 *>(static_cast<uint8_t *>(a.kv) + row * kD)[tid] = make_uint2(w[0], w[1]);
         }
-        if (tid == 0) a.kv_scale[row] = scale;
+        if (tid == 0 && !a.per_tensor) a.kv_scale[row] = scale;
     }
 }
 
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendArgs a) {
 
 int launch_append(const void *c_kv_new, const void *k_pe_new, void *kv_pages, float *kv_scale,
                   const int32_t *page_table, const int32_t *ctx_lens, int B, int T, int num_pages, int max_pages,
-                  int pt_stride, int fp8, int32_t *err, cudaStream_t stream) {
+                  int pt_stride, int fp8, int per_tensor, int32_t *err, cudaStream_t stream) {
     AppendArgs a;
     a.c_kv_new = static_cast<const __nv_bfloat16 *>(c_kv_new);
     a.k_pe_new = static_cast<const __nv_bfloat16 *>(k_pe_new);
@@ -117,6 +119,7 @@ int launch_append(const void *c_kv_new, const void *k_pe_new, void *kv_pages, fl
     a.num_pages = num_pages;
     a.max_pages = max_pages;
     a.pt_stride = pt_stride;
+    a.per_tensor = per_tensor;
     const unsigned grid = (unsigned)((int64_t)B * T);
     if (fp8)
         append_kernel<true><<<grid, kThreads, 0, stream>>>(a);

@@ -40,6 +40,7 @@ struct Problem {
     int B, T, H, R;               // R = T*H query rows per sequence
     int num_pages, max_pages, pt_stride;
     int out_f32;
+    int kv_scale_per_tensor;      // FP8: kv_scale[0] scales every cached value
     int n_slots;                  // KV ranges the global page sequence is cut into
     int n_groups;                 // row groups per sequence
     int rows_per_group;
@@ -243,7 +244,7 @@ __device__ __forceinline__ void store_out(void *out, int64_t idx, float v, int o
 int launch_simt(const Problem &p, cudaStream_t stream);
 int launch_append(const void *c_kv_new, const void *k_pe_new, void *kv_pages, float *kv_scale,
                   const int32_t *page_table, const int32_t *ctx_lens, int B, int T, int num_pages, int max_pages,
-                  int pt_stride, int fp8, int32_t *err, cudaStream_t stream);
+                  int pt_stride, int fp8, int per_tensor, int32_t *err, cudaStream_t stream);
 int launch_tc(const Problem &p, cudaStream_t stream);
 int launch_merge_internal(const Problem &p, cudaStream_t stream);
 int launch_merge_public(const float *out_parts, const float *lse_parts, int n_parts, int64_t rows,

@@ -36,7 +36,7 @@ __device__ __forceinline__ float load_kv(const Problem &p, bool fp8, int64_t row
         const uint8_t *kv = static_cast<const uint8_t *>(p.kv);
         __nv_fp8_e4m3 v;
         v.__x = kv[row * kD + d];
-        return float(v) * __ldg(p.kv_scale + row);
+        return float(v) * __ldg(p.kv_scale + (p.kv_scale_per_tensor ? 0 : row));
     }
     const __nv_bfloat16 *kv = static_cast<const __nv_bfloat16 *>(p.kv);
     return __bfloat162float(kv[row * kD + d]);

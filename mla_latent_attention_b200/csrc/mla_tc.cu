@@ -223,7 +223,9 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
             for (int q = 0; q < C::kParts; ++q) {
                 const int part = q == 0 ? C::kRope : q - 1;
                 if (!waitb(p, ms, &ms.part_empty[stage][part], empty_parity)) return;
-                if (lane == 0) ptx::mbar_arrive_expect_tx(&ms.part_full[stage][part], n_ok * C::part_bytes(part));
+                // a static per-tensor FP8 scale comes with no per-position scale copies
+                const uint32_t pb = C::part_bytes(part) - (kFp8 && part == 0 && p.kv_scale_per_tensor ? 64u : 0u);
+                if (lane == 0) ptx::mbar_arrive_expect_tx(&ms.part_full[stage][part], n_ok * pb);
                 __syncwarp();
                 if (!ok) continue;
                 uint64_t *bar = &ms.part_full[stage][part];
@@ -232,7 +234,7 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                         ptx::tma_load_2d(st + 4 * C::kChunkBytes + lane * 1024, map_b, bar, 512, y);
                     } else {
                         ptx::tma_load_2d(st + part * C::kChunkBytes + lane * 2048, map_a, bar, 128 * part, y);
-                        if (part == 0)
+                        if (part == 0 && !p.kv_scale_per_tensor)
                             ptx::bulk_load(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
                                            p.kv_scale + (int64_t)pid * kPage, 64, bar);
                     }
@@ -573,6 +575,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
     constexpr float kEmpty = -1e30f;           // stabiliser of a row that has seen nothing yet
     uint32_t g = 0;
     GroupSync all_sync(&ms.all_sync), hsync(&ms.half_sync[h]);
+    const float static_scale = kFp8 && p.kv_scale_per_tensor ? __ldg(p.kv_scale) : 1.f;
 
     for_each_piece(p, slot, [&](const Piece &pc) {
         if (aborted(ms)) return;
@@ -652,9 +655,10 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             // value scale of this lane's token; 0 where the slot is not a
             // cached position (its stored scale may be anything, even NaN)
             const float kvs = !kFp8 ? 1.f
-                              : (loaded && pos < pc.ctx)
-                                  ? reinterpret_cast<const float *>(smem + C::kScaleOff + stage * C::kScaleBytes)[i]
-                                  : 0.f;
+                              : !(loaded && pos < pc.ctx) ? 0.f
+                              : p.kv_scale_per_tensor
+                                  ? static_scale
+                                  : reinterpret_cast<const float *>(smem + C::kScaleOff + stage * C::kScaleBytes)[i];
             const float factor = p.sm_scale_log2 * (kFp8 ? kvs * qscale : 1.f);
             const float lkvs = kFp8 ? __log2f(kvs) : 0.f;
             const bool fast = (info & 0xFFu) == 0xFFu && pos0 + kTileM <= min_lim;

@@ -53,6 +53,21 @@ def test_append_bit_exact(kv, T):
         assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_scales.view(np.uint32))
 
 
+def test_append_with_static_scale_bit_exact():
+    """A per-tensor static scale: codes e4m3(x / s), the scale untouched."""
+    w = W.static_scale_workload(W.make_workload("ragged_dcp8", B=4, H=4, ctx_override=("loguniform", 20, 500)))
+    c_new, k_new = _fresh_rows(w.B, w.T, 71, scale=3.0)
+    ref_pages, ref_scales, ok = oracle.append_kv(c_new, k_new, w.kv_pages, w.kv_scale, w.page_table, w.ctx_lens,
+                                                 kv_dtype=W.KV_FP8)
+    assert ok
+    wd = w.to(DEV)
+    pages, scales = wd.kv_pages.clone(), wd.kv_scale.clone()
+    mla.append_kv(c_new.to(DEV), k_new.to(DEV), pages, scales, wd.page_table, wd.ctx_lens)
+    torch.cuda.synchronize()
+    assert np.array_equal(pages.cpu().numpy(), ref_pages)
+    assert np.array_equal(scales.cpu().numpy(), ref_scales)
+
+
 @pytest.mark.parametrize("kv", [W.KV_FP8, W.KV_BF16])
 def test_decode_after_append(kv):
     """Append the drafts' rows, then verify-decode them: GPU append + GPU

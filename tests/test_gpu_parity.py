@@ -144,6 +144,17 @@ def test_context_partitions_merge_to_whole(kernel):
     assert (mo.float() - whole_o.float()).abs().max().item() <= 2e-2 * whole_o.float().abs().max().item()
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("name,kw", [("spec_verify_small", dict(B=3, kv=W.KV_FP8)),
+                                     ("batched_verify_fp8_32k", dict(B=2, ctx_override=("fixed", 3000)))])
+def test_static_fp8_scale_matches_oracle(name, kw, kernel):
+    """A per-tensor static FP8 scale (kv_scale of one element)."""
+    w = W.static_scale_workload(W.make_workload(name, **kw))
+    out, lse = _run(w, kernel)
+    ref_o, ref_l = oracle.decode_workload(w)
+    assert_matches_oracle(out, lse, ref_o, ref_l, w.kv_dtype, f"{name} static scale")
+
+
 # 7 parts: one warp per (row, quarter); 40 parts: eight warps per (row, quarter)
 @pytest.mark.parametrize("n", [7, 40])
 def test_merge_partials_matches_oracle(n):
