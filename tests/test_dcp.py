@@ -70,3 +70,40 @@ def test_dcp_over_cpu_ranks_equals_whole_decode(world, kv):
         # fp32 partials, exact merge: rounding only
         assert err_o <= 1e-6 * scale + 1e-7, (rank, err_o)
         assert err_l <= 1e-5, (rank, err_l)
+
+
+def _rank_dies(rank, world, port, queue):
+    import mla_workloads as W
+    from mla_latent_attention_b200 import dcp
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    w = W.make_workload("spec_verify_small", B=2, H=2, ctx_override=("uniform", 40, 80))
+    part = W.partition_round_robin(w, world)[rank]
+    if rank == 1:
+        os._exit(3)                            # a rank lost before the exchange
+
+    def decode_fn(*args):
+        return torch.zeros((2, 3, 2, 512)), torch.zeros((2, 3, 2))
+
+    try:
+        dcp.dcp_decode(part.q_lat, part.q_pe, part.kv_pages, part.kv_scale, part.page_table, part.ctx_lens,
+                       part.sm_scale, vis_lens=part.vis_lens, decode_fn=decode_fn, merge_fn=lambda o, l, d: (o, l))
+        queue.put((rank, "completed"))
+    except Exception as e:  # the collective must fail, not hang
+        queue.put((rank, type(e).__name__))
+    os._exit(0)
+
+
+def test_dcp_lost_rank_is_an_error_not_a_hang():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies, args=(r, 2, port, queue)) for r in range(2)]
+    for p in procs:
+        p.start()
+    rank, what = queue.get(timeout=90)
+    for p in procs:
+        p.join(timeout=60)
+    assert rank == 0 and what != "completed"
+    assert procs[1].exitcode == 3
