@@ -36,7 +36,7 @@
 //
 // Softmax stabiliser: per query row a running bound m2 on the log2 weight
 // u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
-// the lanes of a row half.  It moves only when some weight exceeds it by more
+// the lanes of a row group.  It moves only when some weight exceeds it by more
 // than TAU (then O^T and the row sums are rescaled), and then to DELTA above
 // the new maximum, so after the first tile it rarely moves again.  Weights
 // are exp2(u - m2 + C), at most 2^(TAU+C), which keeps the e4m3 weights in
@@ -426,7 +426,7 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
 }
 
 // ---------------------------------------------------------------------------
-// warps 2-9: query staging, online softmax, epilogue
+// warps 2-13: query staging, online softmax, epilogue
 // ---------------------------------------------------------------------------
 // Stages the 48 query rows of this group as the score MMA's B operand
 // (K-major, 128B / 64B swizzled chunks).  FP8: one pass into registers, the
@@ -544,7 +544,7 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
     return true;
 }
 
-// 24 rows of one accumulator column block; for FP8 the hi and lo halves
+// kRpt rows of one accumulator column block; for FP8 the hi and lo halves
 // (48 columns apart) are added.
 template <bool kFp8>
 __device__ __forceinline__ void tmem_rows(uint32_t taddr, float *v) {
@@ -567,7 +567,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
     const int w4 = ws & 3;                     // warp within the row group
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int i = quad * 32 + lane;            // tile position / TMEM lane
-    const int st = threadIdx.x - 64;           // 0..255 for cooperative loops
+    const int st = threadIdx.x - 64;           // 0 .. kSoftmaxThreads - 1, for cooperative loops
     const int hst = w4 * 32 + lane;            // 0..127 within the row group
     const int cb = h * kRpt;
     const uint32_t tmem = ms.tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -601,7 +601,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (st == 0 && pc.bad_ctx && g_idx == 0) report_error(p.err, MLA_DEV_BAD_CTX, pc.b);
         if (!all_sync(p, ms)) return;
         const int rows_here = min(kN, p.R - r0);
-        int min_lim = INT_MAX;  // over this half's real rows
+        int min_lim = INT_MAX;  // over this row group's real rows
         for (int c = cb; c < min(cb + kRpt, rows_here); ++c) min_lim = min(min_lim, ms.col_lim[c]);
 
         if (nt == 0) {  // nothing to read: write the empty (or invalid) result
@@ -671,7 +671,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 s[c] = valid ? s[c] * factor : -INFINITY;       // score, log2 units
                 exceed |= s[c] > m2c[c] + kx;
             }
-            // all lanes of the half must agree on the stabiliser
+            // all lanes of the row group must agree on the stabiliser
             const int vote = __any_sync(0xffffffffu, exceed);
             if (lane == 0) ms.vote[h][gg & 1][w4] = vote;
             if (!hsync(p, ms)) return;
@@ -736,8 +736,8 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             }
             unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
             if constexpr (kFp8) {
-                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of the
-                // half.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
+                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of this
+                // thread's rows.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
                 // far below lo's 2^-9), hi = e4m3(p16), and p16 - hi is exact in
                 // f16, so lo = e4m3(p16 - hi).
                 uint32_t hw[kRpt / 4], lw[kRpt / 4];
@@ -804,7 +804,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (!hsync(p, ms)) return;
         const int ncols = min(kRpt, rows_here - cb);
         // O goes out one 128-dim block at a time: every thread writes its dim of
-        // its half's rows into a [48 rows][128] staging box (the query area is
+        // its row group's rows into a [48 rows][128] staging box (the query area is
         // free until the next piece), then one thread stores the box with a
         // tensor store.  The maps clip rows past the sequence's R, and two
         // staging boxes alternate so the next block is written while the
