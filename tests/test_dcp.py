@@ -92,6 +92,9 @@ def _rank_dies(rank, world, port, queue):
         queue.put((rank, "completed"))
     except Exception as e:  # the collective must fail, not hang
         queue.put((rank, type(e).__name__))
+    # os._exit skips the queue's feeder thread: flush the message first
+    queue.close()
+    queue.join_thread()
     os._exit(0)
 
 
