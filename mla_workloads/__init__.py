@@ -320,6 +320,37 @@ def partition_round_robin(w: Workload, n_parts: int, gen_seed: int = 77) -> list
     return parts
 
 
+def ragged_drafts(w: Workload, n_new=None, seed: int = 23) -> Workload:
+    """The same batch with a per-sequence number of query tokens n_new[b] in
+    [1, T] (drawn uniformly unless given), packed into the first n_new[b] of
+    the T query slots.  Sequence b's last n_new[b] cached positions are its
+    new tokens: slot t < n_new[b] sits at position ctx - n_new[b] + t and sees
+    every position up to itself; the remaining slots are padding and see
+    nothing (``vis_lens`` 0).  Returns the workload and n_new."""
+    B, T = w.B, w.T
+    if n_new is None:
+        gen = torch.Generator(device="cpu")
+        gen.manual_seed(seed)
+        n_new = torch.randint(1, T + 1, (B,), generator=gen)
+    n_new = torch.as_tensor(n_new, dtype=torch.int64).cpu()
+    ctx = w.ctx_lens.to("cpu").to(torch.int64)
+    if n_new.shape != (B,) or bool((n_new < 1).any()) or bool((n_new > T).any()) or bool((n_new > ctx).any()):
+        raise ValueError("need 1 <= n_new[b] <= min(T, ctx_lens[b])")
+    t = torch.arange(T).unsqueeze(0)
+    vis = torch.where(t < n_new.unsqueeze(1), ctx.unsqueeze(1) - n_new.unsqueeze(1) + t + 1, 0)
+    return dataclasses.replace(w, vis_lens=vis.to(torch.int32).to(w.ctx_lens.device)), n_new
+
+
+def one_sequence(w: Workload, b: int, T: Optional[int] = None) -> Workload:
+    """Sequence b alone with its first T query slots (default all) and the
+    default causality (no ``vis_lens``); the cache is shared."""
+    T = w.T if T is None else T
+    return dataclasses.replace(w, q_lat=w.q_lat[b:b + 1, :T].contiguous(),
+                               q_pe=w.q_pe[b:b + 1, :T].contiguous(),
+                               page_table=w.page_table[b:b + 1].contiguous(),
+                               ctx_lens=w.ctx_lens[b:b + 1].contiguous(), vis_lens=None)
+
+
 def static_scale_workload(w: Workload) -> Workload:
     """The same FP8 workload re-quantised with one per-tensor scale: the
     dequantised cache values (unused slots stay NaN) divided by

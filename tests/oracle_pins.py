@@ -341,8 +341,27 @@ def pin_static_scale(lib):
             assert np.array_equal(pages[int(ws.page_table[b, pos // 16]), pos % 16], codes[b, t].numpy())
 
 
+def pin_ragged_drafts(lib):
+    """A batch whose sequences carry 1..T query tokens (the rest of the T slots
+    padding, visible count 0) decodes each sequence's real tokens exactly as
+    that sequence decoded alone with its own token count and the default
+    causality; padding rows come out as the empty set: out 0, lse -inf."""
+    for kv in (W.KV_BF16, W.KV_FP8):
+        w0 = _small(kv, T=4, H=2, B=4, ctx=("uniform", 20, 75), seed=29)
+        w, n_new = W.ragged_drafts(w0, n_new=[1, 4, 2, 3])
+        out, lse = oracle.decode_workload(w, lib=lib)
+        out = out.reshape(w.B, w.T, w.H, 512)
+        lse = lse.reshape(w.B, w.T, w.H)
+        for b in range(w.B):
+            k = int(n_new[b])
+            ao, al = oracle.decode_workload(W.one_sequence(w, b, T=k), lib=lib)
+            assert np.array_equal(out[b, :k], ao.reshape(k, w.H, 512)), (kv, b)
+            assert np.array_equal(lse[b, :k], al.reshape(k, w.H)), (kv, b)
+            assert np.all(out[b, k:] == 0.0) and np.all(lse[b, k:] == -np.inf), (kv, b)
+
+
 PINS = [pin_e4m3_table, pin_bf16_widening, pin_library_attention, pin_single_position,
         pin_zero_query, pin_constant_values, pin_two_positions, pin_page_permutation,
         pin_head_padding, pin_split_merge, pin_argmax_recovery, pin_merge_rules,
         pin_e4m3_encode_inverts_decoder, pin_e4m3_encode_rounding, pin_row_quantiser, pin_append_positions,
-        pin_static_scale]
+        pin_static_scale, pin_ragged_drafts]

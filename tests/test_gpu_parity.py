@@ -125,6 +125,26 @@ def test_rows_that_see_nothing(kernel):
     assert_matches_oracle(out, lse, ref_o, ref_l, w.kv_dtype, "empty rows")
 
 
+RAGGED = [
+    ("spec_verify_small", dict(B=5, T=4, ctx_override=("uniform", 200, 1200))),
+    ("batched_verify_fp8_32k", dict(B=4, T=8, ctx_override=("fixed", 700))),
+]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("name,kw", RAGGED, ids=[n for n, _ in RAGGED])
+def test_ragged_draft_depths(name, kw, kernel):
+    """Sequences with 1..T query tokens in one call: real tokens match the
+    oracle, padding slots are the empty set (out 0, lse -inf)."""
+    w, n_new = W.ragged_drafts(W.make_workload(name, **kw))
+    ref_o, ref_l = oracle.decode_workload(w)
+    out, lse = _run(w, kernel)
+    for b in range(w.B):
+        k = int(n_new[b])
+        assert torch.all(out[b, k:] == 0) and torch.all(lse[b, k:].cpu() == -float("inf")), b
+    assert_matches_oracle(out, lse, ref_o, ref_l, w.kv_dtype, f"ragged {name}/{kernel}")
+
+
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_context_partitions_merge_to_whole(kernel):
     """Round-robin 8-way context partitions, each decoded to fp32 partials,
