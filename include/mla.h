@@ -24,6 +24,9 @@
  * work", section 1, multi-token verification #51705); token t sits at
  * position ctx - T + t and sees positions 0 .. ctx - T + t, i.e.
  * n = ctx_lens[b] - T + t + 1, unless mla_dims.vis_lens gives n explicitly.
+ * vis_lens also carries a batch whose sequences have different draft depths:
+ * a sequence with k < T tokens puts them in slots 0..k-1 with
+ * n = ctx_lens[b] - k + t + 1 and gives the unused slots n = 0.
  *
  * Long histories are split across the GPU's SMs and the partial answers are
  * merged exactly through their log-sum-exp normalisers ("Inside Kimi K3
