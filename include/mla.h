@@ -150,6 +150,10 @@ MLA_API int64_t mla_decode_workspace_size(const mla_dims *dims);
  *                                   (whose out is then 0).  May be NULL.
  *   workspace  device scratch of at least mla_decode_workspace_size(dims)
  *              bytes, 256-byte aligned.  Not shared between calls in flight.
+ *              Its first 8 bytes are the sticky device error word, which
+ *              mla_decode only ever sets: clear it once before the first call
+ *              (mla_reset_device_error, or zero the whole workspace) if it is
+ *              going to be read with mla_read_device_error.
  *
  * Rows with no visible position (only possible with vis_lens) produce out = 0
  * and lse = -inf, the identity of the merge below.

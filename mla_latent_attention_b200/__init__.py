@@ -153,7 +153,9 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, o
     """Paged MLA decode (``mla_decode``).  Returns (out [B,T,H,512], lse [B,T,H] fp32).
 
     ``stage_event`` (a ``torch.cuda.Event``) is recorded between the attention
-    kernel and the merge kernel, for timing the two apart."""
+    kernel and the merge kernel, for timing the two apart.  A ``workspace``
+    whose device error word will be read (``read_device_error``) must start
+    zeroed (``torch.zeros``, or ``reset_device_error`` once)."""
     lib = load_library()
     dev = q_lat.device
     B, T, H = q_lat.shape[:3]
