@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-append", dest="append", action="store_false",
+                    help="skip timing the cache writer (mla_append_kv) on the workload's new tokens")
     return ap.parse_args()
 
 
@@ -278,6 +280,45 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
+def time_append(mla, w, kv, sc, L, stream, reps=50):
+    """The cache writer on its own: each layer's T new tokens per sequence
+    written (and, for an FP8 cache, quantised) by one mla_append_kv, the L
+    launches captured as a graph and replayed ``reps`` times."""
+    dev = w.q_lat.device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(31)
+    c_new = torch.randn((w.B, w.T, W.D_LATENT), generator=gen, device=dev).to(torch.bfloat16)
+    k_new = torch.randn((w.B, w.T, W.D_ROPE), generator=gen, device=dev).to(torch.bfloat16)
+
+    def step():
+        for i in range(L):
+            mla.append_kv(c_new, k_new, kv[i], None if sc is None else sc[i], w.page_table, w.ctx_lens)
+
+    step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            step()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (reps * L)
+    tokens = w.B * w.T
+    # bf16 values in; FP8 codes plus the token's scale, or bf16 values, out
+    out_bytes = W.D_QK + 4 if w.kv_dtype == W.KV_FP8 else 2 * W.D_QK
+    nbytes = tokens * (2 * W.D_QK + out_bytes)
+    return {"us_per_launch": us, "tokens_per_launch": tokens, "bytes_per_launch": nbytes,
+            "achieved_gbs": nbytes / us / 1e3, "launches": reps * L,
+            "note": "one launch per layer, timed apart from the decode step"}
+
+
 def run_ours(args, rank, world, local_rank):
     import mla_latent_attention_b200 as mla
     dev = torch.device("cuda", local_rank)
@@ -399,6 +440,9 @@ def run_ours(args, rank, world, local_rank):
     h2d = (h_qlat.numel() * h_qlat.element_size() + h_qpe.numel() * h_qpe.element_size())
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
 
+    # after every decode measurement: the writer changes the caches' last T slots
+    append = time_append(mla, w, kv, sc, L, stream) if args.append else None
+
     if rank != 0:
         return
     peaks, peak_src = load_peaks()
@@ -435,6 +479,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": steps * L * launches_per_call,
         "clocks": clocks,
     }
+    if append is not None:
+        line["append"] = append
     if world == 1 and not args.no_cpu_baseline:
         st, rows, spent, threads = oracle_sample(w, L, args.cpu_seconds)
         line["cpu_baseline"] = {
