@@ -133,6 +133,15 @@ def step_units(w, layers):
                 seqs=w.B)
 
 
+def workload_config(args, w, units, kernel, parallelism):
+    """The bench line's ``config``: the same keys for both arms."""
+    return {"workload": args.workload, "B": w.B, "T": w.T, "H": w.H, "ctx": int(w.ctx_lens.max()),
+            "kv": w.kv_dtype, "layers": args.layers, "kernel": kernel, "num_splits": args.num_splits,
+            "parallelism": parallelism,
+            "l2": f"inputs larger than L2: {args.layers} layer caches, "
+                  f"{units['kv_bytes'] / 1e9:.2f} GB of KV per step"}
+
+
 _LIBCUDA = None
 
 
@@ -266,8 +275,7 @@ def run_reference(args, rank, world):
         "steps": steps, "warmup": args.warmup, "ms_per_step": step_time * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": args.workload, "B": w.B, "T": w.T, "H": w.H, "kv": w.kv_dtype,
-                   "layers": args.layers},
+        "config": workload_config(args, w, units, "oracle", "oracle on host cores"),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"{rows} whole query rows of one layer per step "
                                    f"({spent:.1f} s), extrapolated to {args.layers} layers x "
@@ -464,12 +472,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": max_elapsed / steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": kernel_dtype, "data": "synthetic",
-        "config": {"workload": args.workload, "B": B, "T": T, "H": H,
-                   "ctx": int(w.ctx_lens.max()), "kv": w.kv_dtype, "layers": L,
-                   "kernel": args.kernel, "num_splits": args.num_splits,
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {L} layer caches, "
-                         f"{units['kv_bytes'] / 1e9:.2f} GB of KV per step"},
+        "config": workload_config(args, w, units, args.kernel, f"replicas x{world}"),
         "hbm_fraction_of_8TBs": value / world / NOMINAL_HBM_GBS,
         "seq_steps_per_s": world * steps * units["seqs"] / max_elapsed,
         "tensor_tflops": tflops,
