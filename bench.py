@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_ctx_142k", choices=W.CONFIG_ORDER)
     ap.add_argument("--kv", choices=[W.KV_BF16, W.KV_FP8], default=None)
+    ap.add_argument("--T", type=int, default=None, help="query tokens per sequence (1 + drafts), 1..8")
+    ap.add_argument("--static-scale", action="store_true",
+                    help="FP8 cache with one per-tensor scale instead of one per position")
     ap.add_argument("--layers", type=int, default=24)
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05"])
     ap.add_argument("--num-splits", type=int, default=0)
@@ -110,6 +113,13 @@ def recorded_traffic(workload: str, kv: str):
     return None
 
 
+def make_bench_workload(args, device="cpu"):
+    w = W.make_workload(args.workload, device=device, kv=args.kv, T=args.T)
+    if args.static_scale:
+        w = W.static_scale_workload(w)
+    return w
+
+
 def visible_positions(w) -> int:
     """Sum over query rows' distinct sequences of cached positions read once
     per layer (each sequence's pages are read once for all its rows)."""
@@ -136,7 +146,7 @@ def step_units(w, layers):
 def workload_config(args, w, units, kernel, parallelism):
     """The bench line's ``config``: the same keys for both arms."""
     return {"workload": args.workload, "B": w.B, "T": w.T, "H": w.H, "ctx": int(w.ctx_lens.max()),
-            "kv": w.kv_dtype, "layers": args.layers, "kernel": kernel, "num_splits": args.num_splits,
+            "kv": w.kv_label(), "layers": args.layers, "kernel": kernel, "num_splits": args.num_splits,
             "parallelism": parallelism,
             "l2": f"inputs larger than L2: {args.layers} layer caches, "
                   f"{units['kv_bytes'] / 1e9:.2f} GB of KV per step"}
@@ -256,7 +266,7 @@ def oracle_sample(w, layers, seconds):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = W.make_workload(args.workload, kv=args.kv)
+    w = make_bench_workload(args)
     units = step_units(w, args.layers)
     steps = args.steps if args.steps is not None else 3
     budget = max(0.5, 120.0 / (steps + args.warmup))   # whole run within ~2 minutes
@@ -319,8 +329,8 @@ def time_append(mla, w, kv, sc, L, stream, reps=50):
     torch.cuda.synchronize()
     us = a.elapsed_time(b) * 1e3 / (reps * L)
     tokens = w.B * w.T
-    # bf16 values in; FP8 codes plus the token's scale, or bf16 values, out
-    out_bytes = W.D_QK + 4 if w.kv_dtype == W.KV_FP8 else 2 * W.D_QK
+    # bf16 values in; the stored form out (FP8 codes and, per position, the scale; or bf16)
+    out_bytes = w.kv_bytes_per_position()
     nbytes = tokens * (2 * W.D_QK + out_bytes)
     return {"us_per_launch": us, "tokens_per_launch": tokens, "bytes_per_launch": nbytes,
             "achieved_gbs": nbytes / us / 1e3, "launches": reps * L,
@@ -331,7 +341,7 @@ def run_ours(args, rank, world, local_rank):
     import mla_latent_attention_b200 as mla
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = W.make_workload(args.workload, device=dev, kv=args.kv)
+    w = make_bench_workload(args, device=dev)
     L = args.layers
     units = step_units(w, L)
     # each layer: its own copy of the paged cache (same contents, own memory)
@@ -461,7 +471,7 @@ def run_ours(args, rank, world, local_rank):
     achieved_gbs = per_launch_bytes / dec_avg / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak, "traffic": recorded_traffic(args.workload, w.kv_dtype),
+                "frac": achieved_gbs / hbm_peak, "traffic": recorded_traffic(args.workload, w.kv_label()),
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "kernel": "mla decode attention kernel", "peak_source": f"{peak_src} hbm_gbs",
                 "avg_launch_us": dec_avg * 1e6, "merge_avg_launch_us": sum(mer) / len(mer) * 1e6}

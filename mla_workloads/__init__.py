@@ -122,7 +122,16 @@ class Workload:
         return int(self.ctx_lens.to(torch.int64).sum())
 
     def kv_bytes_per_position(self) -> int:
-        return D_QK * 2 if self.kv_dtype == KV_BF16 else D_QK + 4
+        """bf16: 1,152; FP8: 576 codes + a 4-byte scale, or 576 with one static scale."""
+        if self.kv_dtype == KV_BF16:
+            return D_QK * 2
+        return D_QK if self.kv_scale is not None and self.kv_scale.numel() == 1 else D_QK + 4
+
+    def kv_label(self) -> str:
+        """Cache format: "bf16", "fp8" (per-position scales) or "fp8-static"."""
+        if self.kv_dtype == KV_FP8 and self.kv_scale is not None and self.kv_scale.numel() == 1:
+            return KV_FP8 + "-static"
+        return self.kv_dtype
 
 
 DEFAULT_SM_SCALE = 1.0 / math.sqrt(192.0)

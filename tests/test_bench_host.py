@@ -98,3 +98,24 @@ def test_reference_arm_line():
     assert set(line["config"]) == set(ours)
     for k in ("workload", "B", "T", "H", "ctx", "kv", "layers", "l2"):
         assert line["config"][k] == ours[k], k
+
+
+def test_step_units_static_scale_and_depth():
+    """One static FP8 scale: 576 B per position (no per-position scale);
+    --T changes the number of query tokens and so the flops."""
+    w = W.make_workload("long_ctx_142k", ctx_override=("fixed", 640), T=4)
+    ws = W.static_scale_workload(w)
+    assert ws.kv_label() == "fp8-static" and w.kv_label() == "fp8"
+    u = bench.step_units(ws, 2)
+    assert u["kv_bytes"] == 640 * 576 * 2
+    assert u["flops"] == 2176 * 96 * sum(640 - 4 + t + 1 for t in range(4)) * 2
+
+
+def test_reference_arm_static_scale_and_depth():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "spec_verify_small", "--kv", "fp8", "--static-scale", "--T", "5",
+                        "--layers", "1", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["config"]["T"] == 5 and line["config"]["kv"] == "fp8-static" and line["value"] > 0
