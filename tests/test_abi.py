@@ -111,3 +111,50 @@ def test_status_strings(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(mla.MlaError):
         mla.load_library(str(tmp_path / "missing.so"))
+
+
+_LAYOUT_PROBE = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "mla.h"
+#define F(name) printf("%s %zu\n", #name, offsetof(mla_dims, name));
+int main(void) {
+    printf("sizeof %zu\n", sizeof(mla_dims));
+    F(B) F(T) F(H) F(num_pages) F(max_pages_per_seq) F(page_table_stride) F(kv_dtype)
+    F(out_dtype) F(num_splits) F(kernel) F(vis_lens) F(stage_event) F(kv_scale_per_tensor)
+    return 0;
+}
+"""
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c99"), ("g++", "-std=c++17")])
+def test_header_compiles_standalone(tmp_path, compiler, std):
+    """include/mla.h is plain C: it compiles on its own with warnings as errors."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not available")
+    src = tmp_path / ("probe.c" if compiler == "gcc" else "probe.cpp")
+    src.write_text(_LAYOUT_PROBE)
+    r = subprocess.run([compiler, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), str(src), "-o", str(tmp_path / "probe")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_binding_struct_matches_header_layout(tmp_path):
+    """The ctypes mirror of mla_dims has the header's size and field offsets."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "probe.c"
+    src.write_text(_LAYOUT_PROBE)
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    c = dict(line.split() for line in out if line)
+    assert int(c.pop("sizeof")) == ctypes.sizeof(mla.Dims)
+    assert list(c) == [f[0] for f in mla.Dims._fields_]
+    for name, off in c.items():
+        assert getattr(mla.Dims, name).offset == int(off), name
