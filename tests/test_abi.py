@@ -158,3 +158,23 @@ def test_binding_struct_matches_header_layout(tmp_path):
     assert list(c) == [f[0] for f in mla.Dims._fields_]
     for name, off in c.items():
         assert getattr(mla.Dims, name).offset == int(off), name
+
+
+def _prototypes():
+    """{name: number of parameters} of every MLA_API function in include/*.h."""
+    protos = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = re.sub(r"/\*.*?\*/", " ", open(h).read(), flags=re.S)
+        for name, params in re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(([^)]*)\)\s*;", src):
+            params = params.strip()
+            protos[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_argument_counts_match_prototypes(lib):
+    protos = _prototypes()
+    assert set(protos) == _declared()
+    for name, n in protos.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, f"{name}: the binding sets no argtypes"
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
