@@ -71,7 +71,7 @@ typedef struct CUstream_st *mla_stream_t;
 typedef enum {
     MLA_OK = 0,
     MLA_ERR_INVALID_ARG = -1,  /* null pointer, non-positive size, bad enum, misalignment */
-    MLA_ERR_UNSUPPORTED = -2,  /* valid request this build cannot run (e.g. no sm_100 device) */
+    MLA_ERR_UNSUPPORTED = -2,  /* valid request the library cannot run here (e.g. no sm_100 device) */
     MLA_ERR_WORKSPACE = -3,    /* workspace missing, misaligned or smaller than required */
     MLA_ERR_CUDA = -4          /* a CUDA runtime/driver call failed; see mla_last_cuda_error */
 } mla_status;
