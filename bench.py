@@ -143,6 +143,16 @@ def step_units(w, layers):
                 seqs=w.B)
 
 
+def max_over_ranks(seconds: float, world: int, device) -> float:
+    """The largest of every rank's time (each rank passes its own); the
+    value itself with one rank.  Every rank must call it at the same point."""
+    if world <= 1:
+        return float(seconds)
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_config(args, w, units, kernel, parallelism):
     """The bench line's ``config``: the same keys for both arms."""
     return {"workload": args.workload, "B": w.B, "T": w.T, "H": w.H, "ctx": int(w.ctx_lens.max()),
@@ -426,10 +436,7 @@ def run_ours(args, rank, world, local_rank):
         mer += [event_ms(ev_m[i], ev_b[i]) / 1e3 for i in range(L)]
     clocks = sampler.stop()
 
-    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_elapsed = float(t.item())
+    max_elapsed = max_over_ranks(elapsed, world, dev)
 
     # end to end through the public API with host buffers: per step the query
     # rows of every layer go host->device and the outputs come back.
@@ -451,10 +458,8 @@ def run_ours(args, rank, world, local_rank):
         h_lse.copy_(lses, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_t = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = world * e2e_steps * units["kv_bytes"] / float(e2e_t.item()) / 1e9
+    e2e_time = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    e2e_value = world * e2e_steps * units["kv_bytes"] / e2e_time / 1e9
     h2d = (h_qlat.numel() * h_qlat.element_size() + h_qpe.numel() * h_qpe.element_size())
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
 

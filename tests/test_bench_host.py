@@ -1,6 +1,7 @@
 """Host-side bookkeeping of bench.py (CPU only): the algorithmic units a step
 is credited with, the comment-blind kernel hash that gates the recorded DRAM
-traffic, and the reference arm's JSON line."""
+traffic, the reference arm's JSON line, and the multi-rank path (max over
+ranks on two gloo ranks; the reference arm under torchrun with two ranks)."""
 import json
 import os
 import shutil
@@ -119,3 +120,56 @@ def test_reference_arm_static_scale_and_depth():
     assert r.returncode == 0, r.stderr[-2000:]
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["config"]["T"] == 5 and line["config"]["kv"] == "fp8-static" and line["value"] > 0
+
+
+def _max_rank(rank, world, port, queue):
+    import datetime
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        queue.put((rank, bench.max_over_ranks(1.5 + rank, world, "cpu")))
+    finally:
+        dist.destroy_process_group()
+    queue.close()
+    queue.join_thread()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    """The timed region's duration is the slowest rank's, on every rank."""
+    import multiprocessing as mp
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    procs = [ctx.Process(target=_max_rank, args=(r, 2, port, queue)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(queue.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == {0: 2.5, 1: 2.5}
+    assert bench.max_over_ranks(0.25, 1, "cpu") == 0.25
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Launched like the multi-GPU bench (torchrun, 2 ranks): rank 0 alone
+    runs the oracle and prints one line; both ranks exit 0."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port),
+                        os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "single_query_256", "--layers", "1", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["value"] > 0
