@@ -40,12 +40,11 @@
 // than TAU (then O^T and the row sums are rescaled), and then to DELTA above
 // the new maximum, so after the first tile it rarely moves again.  Weights
 // are exp2(u - m2 + C), at most 2^(TAU+C), which keeps the e4m3 weights in
-// range.  Row sums are kept per lane and reduced once per
-// piece.
+// range.  Row sums are kept per lane and reduced once per piece.
 //
-// Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA records a timeout in the
-// error word, stops, drains its outstanding copies and MMAs and frees its
-// tensor memory.
+// Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA
+// records a timeout in the error word, stops, drains its outstanding copies
+// and MMAs and frees its tensor memory.
 #include <cuda.h>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
