@@ -337,17 +337,27 @@ int oracle_mla_decode(int B, int T, int H, const uint16_t *q_lat, const uint16_t
  *   L = max_i lse_i,  w_i = exp(lse_i - L),  out = sum_i w_i out_i / sum_i w_i,
  *   lse = L + ln sum_i w_i.
  * Parts with lse = -inf weigh nothing; if every part is -inf the row is empty:
- * out = 0, lse = -inf.  out_parts: [n_parts, rows, dv]; lse_parts: [n_parts, rows]. */
+ * out = 0, lse = -inf.  A NaN lse in any part makes the row NaN (out and lse).
+ * out_parts: [n_parts, rows, dv]; lse_parts: [n_parts, rows]. */
 int oracle_mla_merge(int n_parts, int64_t rows, int dv, const double *out_parts,
                      const double *lse_parts, double *out, double *lse) {
     if (n_parts <= 0 || rows < 0 || dv <= 0) return -1;
     for (int64_t r = 0; r < rows; ++r) {
         double L = -INFINITY;
+        int poisoned = 0;
         for (int i = 0; i < n_parts; ++i) {
             double l = lse_parts[(int64_t)i * rows + r];
-            if (l > L) L = l;
+            if (isnan(l)) poisoned = 1;
+            else if (l > L) L = l;
         }
         double *o = out + r * dv;
+        /* a NaN normaliser (a part computed from invalid input) poisons the row,
+           also when every part is NaN and no maximum exists */
+        if (poisoned) {
+            for (int d = 0; d < dv; ++d) o[d] = NAN;
+            lse[r] = NAN;
+            continue;
+        }
         for (int d = 0; d < dv; ++d) o[d] = 0.0;
         if (L == -INFINITY) {
             lse[r] = -INFINITY;

@@ -219,7 +219,8 @@ def pin_argmax_recovery(lib):
 
 
 def pin_merge_rules(lib):
-    """Merge: one part is the identity; -inf parts weigh nothing; all -inf is empty."""
+    """Merge: one part is the identity; -inf parts weigh nothing; all -inf is
+    empty; equal normalisers average; a NaN normaliser poisons its row."""
     rng = np.random.default_rng(4)
     o = rng.standard_normal((1, 5, 8))
     l = rng.standard_normal((1, 5))
@@ -235,6 +236,14 @@ def pin_merge_rules(lib):
     l3 = np.zeros((2, 5))
     mo, ml = oracle.merge(o2, l3, lib=lib)
     assert np.allclose(mo, o2.mean(0), rtol=1e-14) and np.allclose(ml, math.log(2.0), rtol=1e-15)
+    # a NaN normaliser poisons its row only, also when every part of it is NaN
+    l4 = np.zeros((2, 5))
+    l4[1, 1] = np.nan
+    l4[:, 3] = np.nan
+    mo, ml = oracle.merge(o2, l4, lib=lib)
+    assert np.isnan(mo[[1, 3]]).all() and np.isnan(ml[[1, 3]]).all()
+    ok = [0, 2, 4]
+    assert np.allclose(mo[ok], o2.mean(0)[ok], rtol=1e-14) and np.isfinite(ml[ok]).all()
 
 
 def pin_e4m3_encode_inverts_decoder(lib):

@@ -193,12 +193,16 @@ def test_merge_partials_matches_oracle(n):
     fin = np.isfinite(ref_l)
     assert np.abs(got_o - ref_o).max() <= 1e-5 * np.abs(ref_o).max()
     assert np.abs(got_l[fin] - ref_l[fin]).max() <= 1e-5
-    # a NaN normaliser poisons its row
+    # a NaN normaliser poisons its row, also when every part of the row is NaN
     l2 = l.clone()
     l2[4, 9] = float("nan")
+    l2[:, 11] = float("nan")
     mo, ml = mla.merge_partials(o.float().to(DEV), l2.float().to(DEV))
     torch.cuda.synchronize()
     assert torch.isnan(mo[9].float()).all() and torch.isnan(ml[9])
+    assert torch.isnan(mo[11].float()).all() and torch.isnan(ml[11])
+    _, ref_l2 = oracle.merge(o.numpy(), l2.numpy())
+    assert np.array_equal(np.isnan(ml.double().cpu().numpy()), np.isnan(ref_l2))
 
 
 @pytest.mark.parametrize("kernel", KERNELS)

@@ -46,6 +46,7 @@ MUTANTS = {
     "append_position_shifted": ("int pos = ctx - T + t;", "int pos = ctx - T + t + 1;"),
     "append_drops_rope": ("memcpy(row + ORACLE_DL, k_pe_new", "memset(row + ORACLE_DL, 0, 1); (void)(k_pe_new"),
     "empty_row_lse_zero": ("*lse = -INFINITY;\n        return 0;", "*lse = 0.0;\n        return 0;"),
+    "merge_nan_not_checked": ("if (poisoned) {", "if (0) {"),
     "vis_lens_transposed": ("return p->vis_lens[(int64_t)b * p->T + t];", "return p->vis_lens[(int64_t)t * p->B + b];"),
 }
 
