@@ -245,10 +245,16 @@ def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, d
     B, T = int(c_kv_new.shape[0]), int(c_kv_new.shape[1])
     _need(c_kv_new, "c_kv_new", torch.bfloat16, dev, (B, T, 512))
     _need(k_pe_new, "k_pe_new", torch.bfloat16, dev, (B, T, 64))
+    _need(kv_pages, "kv_pages", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), dev)
+    if kv_pages.dim() != 3 or kv_pages.shape[1:] != (16, 576):
+        raise MlaError(f"kv_pages must be [P,16,576], got {tuple(kv_pages.shape)}")
     _need(page_table, "page_table", torch.int32, dev)
+    if page_table.dim() != 2 or page_table.shape[0] != B or page_table.stride(1) != 1:
+        raise MlaError("page_table must be [B, max_pages] int32 with unit column stride")
     _need(ctx_lens, "ctx_lens", torch.int32, dev, (B,))
-    if kv_scale is not None:
-        _need(kv_scale, "kv_scale", torch.float32, dev)
+    if kv_scale is not None:  # per position [P,16] (written), or one static scale (read)
+        _need(kv_scale, "kv_scale", torch.float32, dev,
+              (1,) if kv_scale.numel() == 1 else (kv_pages.shape[0], 16))
     if device_error is not None:
         _need(device_error, "device_error", torch.int32, dev, (2,))
     dims = Dims(B=B, T=T, H=1, num_pages=int(kv_pages.shape[0]), max_pages_per_seq=int(page_table.shape[1]),

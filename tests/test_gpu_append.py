@@ -119,3 +119,13 @@ def test_append_host_errors():
     with pytest.raises(mla.MlaError):        # wrong shape
         mla.append_kv(c_new[:, :, :256].contiguous().to(DEV), k_new.to(DEV), w.kv_pages, None, w.page_table,
                       w.ctx_lens)
+    w8 = W.make_workload("spec_verify_small", B=1, T=1, kv=W.KV_FP8, ctx_override=("fixed", 40)).to(DEV)
+    with pytest.raises(mla.MlaError):        # one scale per page instead of per position
+        mla.append_kv(c_new.to(DEV), k_new.to(DEV), w8.kv_pages, w8.kv_scale[:, 0].contiguous(), w8.page_table,
+                      w8.ctx_lens)
+    with pytest.raises(mla.MlaError):        # page table of another batch size
+        mla.append_kv(c_new.to(DEV), k_new.to(DEV), w8.kv_pages, w8.kv_scale, w8.page_table.repeat(2, 1),
+                      w8.ctx_lens)
+    with pytest.raises(mla.MlaError):        # pages not [P,16,576]
+        mla.append_kv(c_new.to(DEV), k_new.to(DEV), w8.kv_pages.view(-1, 576), w8.kv_scale, w8.page_table,
+                      w8.ctx_lens)
