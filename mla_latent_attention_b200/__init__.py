@@ -187,8 +187,10 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, o
     need = workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    elif workspace.numel() * workspace.element_size() < need:
-        raise MlaError(f"workspace has {workspace.numel()} bytes, needs {need}")
+    else:
+        _need(workspace, "workspace", None, dev)
+        if workspace.numel() * workspace.element_size() < need:
+            raise MlaError(f"workspace has {workspace.numel() * workspace.element_size()} bytes, needs {need}")
     rc = lib.mla_decode(_ptr(q_lat), _ptr(q_pe), _ptr(kv_pages), _ptr(kv_scale), _ptr(page_table),
                         _ptr(ctx_lens), float(sm_scale), _ptr(out), _ptr(lse), ctypes.byref(dims),
                         _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -225,6 +227,8 @@ def merge_partials(out_parts, lse_parts, *, out=None, lse=None, out_dtype=torch.
         _need(out, "out", (torch.bfloat16, torch.float32), dev, (*rows_shape, 512))
     if lse is None:
         lse = torch.empty(rows_shape, dtype=torch.float32, device=dev)
+    else:
+        _need(lse, "lse", torch.float32, dev, rows_shape)
     rc = lib.mla_merge_partials(_ptr(out_parts), _ptr(lse_parts), int(n), rows, _ptr(out),
                                 OUT_F32 if out.dtype == torch.float32 else OUT_BF16, _ptr(lse),
                                 _stream(stream, dev))
@@ -268,6 +272,7 @@ def append_kv(c_kv_new, k_pe_new, kv_pages, kv_scale, page_table, ctx_lens, *, d
 
 def read_device_error(workspace, stream=None):
     """(code, info) of the workspace error word; synchronises the stream."""
+    _need(workspace, "workspace")
     code, info = ctypes.c_int32(0), ctypes.c_int32(0)
     rc = load_library().mla_read_device_error(_ptr(workspace), ctypes.byref(code), ctypes.byref(info),
                                               _stream(stream, workspace.device))
@@ -276,5 +281,6 @@ def read_device_error(workspace, stream=None):
 
 
 def reset_device_error(workspace, stream=None):
+    _need(workspace, "workspace")
     rc = load_library().mla_reset_device_error(_ptr(workspace), _stream(stream, workspace.device))
     _check(rc, "mla_reset_device_error")
