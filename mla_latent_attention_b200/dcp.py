@@ -46,8 +46,8 @@ def dcp_decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, 
 
     Arguments are those of ``mla_latent_attention_b200.decode`` for this
     rank's subset (``vis_lens`` [B,T]: how many of this rank's positions each
-    query token sees).  Returns (out [B,T,H,512] out_dtype, lse [B,T,H] fp32),
-    the same on every rank."""
+    query token sees); every rank passes the same query rows.  Returns
+    (out [B,T,H,512] out_dtype, lse [B,T,H] fp32), the same on every rank."""
     decode_fn = decode_fn or _gpu_decode
     merge_fn = merge_fn or _gpu_merge
     world = dist.get_world_size(group)
@@ -68,7 +68,8 @@ def dcp_decode_sharded(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm
     Gathers the queries of all heads, decodes them over this rank's positions
     (the other arguments as for ``dcp_decode``), exchanges the fp32 partials
     all-to-all by head, and merges the N partials of this rank's heads.
-    Returns (out [B,T,Hl,512] out_dtype, lse [B,T,Hl] fp32)."""
+    Every rank must pass the same B, T and Hl (the collectives move equal
+    blocks).  Returns (out [B,T,Hl,512] out_dtype, lse [B,T,Hl] fp32)."""
     decode_fn = decode_fn or _gpu_decode
     merge_fn = merge_fn or _gpu_merge
     world = dist.get_world_size(group)
