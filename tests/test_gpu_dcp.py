@@ -1,6 +1,7 @@
 """Context-parallel decode through the library on one GPU: a one-rank NCCL
-group (the exchange is then a copy) around the CUDA decode and merge, against
-the oracle's whole-cache decode.  The multi-rank exchange itself is covered
+group (the exchange is then a copy) around the CUDA decode and merge, in both
+forms (partials all-gathered; heads sharded with an all-to-all), against the
+oracle's whole-cache decode.  The multi-rank exchange itself is covered
 on CPU ranks (test_dcp.py)."""
 import datetime
 import socket
@@ -33,5 +34,12 @@ def test_dcp_one_rank_nccl():
         torch.cuda.synchronize()
         ref_o, ref_l = oracle.decode_workload(w)
         assert_matches_oracle(out, lse, ref_o, ref_l, w.kv_dtype, "dcp one rank")
+        # the head-sharded form: with one rank it owns every head
+        out_s, lse_s = dcp.dcp_decode_sharded(part.q_lat, part.q_pe, part.kv_pages, part.kv_scale,
+                                              part.page_table, part.ctx_lens, part.sm_scale,
+                                              vis_lens=part.vis_lens)
+        torch.cuda.synchronize()
+        assert tuple(out_s.shape) == tuple(out.shape) and tuple(lse_s.shape) == tuple(lse.shape)
+        assert_matches_oracle(out_s, lse_s, ref_o, ref_l, w.kv_dtype, "head-sharded dcp one rank")
     finally:
         dist.destroy_process_group()
