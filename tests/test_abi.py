@@ -58,7 +58,9 @@ def _dims(**kw):
 
 BAD_DIMS = [dict(B=0), dict(T=0), dict(T=9), dict(H=0), dict(T=8, H=129), dict(num_pages=0),
             dict(max_pages_per_seq=0), dict(page_table_stride=8), dict(kv_dtype=2),
-            dict(out_dtype=5), dict(num_splits=-1), dict(kernel=7)]
+            dict(out_dtype=5), dict(num_splits=-1), dict(kernel=7),
+            dict(B=1 << 26, T=8, H=1),                 # 2^29 query rows: past the merge grid
+            dict(kv_scale_per_tensor=2), dict(kv_scale_per_tensor=1)]  # the latter with a bf16 cache
 
 
 @pytest.mark.parametrize("bad", BAD_DIMS, ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))

@@ -125,6 +125,17 @@ def test_rows_that_see_nothing(kernel):
     assert_matches_oracle(out, lse, ref_o, ref_l, w.kv_dtype, "empty rows")
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("kv", [W.KV_FP8, W.KV_BF16])
+def test_most_query_rows_per_sequence(kv, kernel):
+    """T * H = 8 * 128 = 1024 query rows per sequence, the most a call takes:
+    22 row groups of 48 for the tensor-core kernel, the last one partial."""
+    w = W.make_workload("batched_verify_fp8_32k", B=2, T=8, H=128, kv=kv, ctx_override=("uniform", 300, 700))
+    ref_o, ref_l = oracle.decode_workload(w)
+    out, lse = _run(w, kernel)
+    assert_matches_oracle(out, lse, ref_o, ref_l, w.kv_dtype, f"1024 rows {kv}/{kernel}")
+
+
 RAGGED = [
     ("spec_verify_small", dict(B=5, T=4, ctx_override=("uniform", 200, 1200))),
     ("batched_verify_fp8_32k", dict(B=4, T=8, ctx_override=("fixed", 700))),
