@@ -176,6 +176,28 @@ def test_context_partitions_merge_to_whole(kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+def test_partitions_holding_none_of_a_sequence(kernel):
+    """Sequences shorter than the partition count: some partitions hold none
+    of their positions (no pages, visible count 0) and must return the empty
+    result, out 0 and lse -inf, which the merge then ignores."""
+    w = W.make_workload("ragged_dcp8", B=4, H=8, ctx_override=("uniform", 3, 12))
+    ref_o, ref_l = oracle.decode_workload(w)
+    parts = W.partition_round_robin(w, 8)
+    empty = [(k, b) for k, p in enumerate(parts) for b in range(w.B) if int(p.ctx_lens[b]) == 0]
+    assert empty
+    outs, lses = [], []
+    for p in parts:
+        o, l = _run(p, kernel, out_dtype=torch.float32)
+        outs.append(o)
+        lses.append(l)
+    for k, b in empty:
+        assert torch.all(outs[k][b] == 0) and torch.all(lses[k][b].cpu() == -float("inf")), (k, b)
+    mo, ml = mla.merge_partials(torch.stack(outs), torch.stack(lses))
+    torch.cuda.synchronize()
+    assert_matches_oracle(mo, ml, ref_o, ref_l, w.kv_dtype, "partitions with empty sequences")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("name,kw", [("spec_verify_small", dict(B=3, kv=W.KV_FP8)),
                                      ("batched_verify_fp8_32k", dict(B=2, ctx_override=("fixed", 3000)))])
 def test_static_fp8_scale_matches_oracle(name, kw, kernel):
