@@ -110,6 +110,23 @@ def test_append_device_errors():
     assert err.tolist() == [1, 2]             # MLA_DEV_BAD_PAGE, sequence 2
 
 
+def test_append_through_padded_page_table():
+    """Page-table rows inside a wider array (row stride larger than the row)
+    place the tokens exactly as the contiguous table does."""
+    w = W.make_workload("spec_verify_small", B=3, kv=W.KV_FP8, ctx_override=("uniform", 60, 300))
+    c_new, k_new = _fresh_rows(w.B, w.T, 83)
+    wd = w.to(DEV)
+    B, n = w.page_table.shape
+    wide = torch.full((B, n + 5), -1, dtype=torch.int32, device=DEV)
+    wide[:, :n] = wd.page_table
+    p1, s1 = wd.kv_pages.clone(), wd.kv_scale.clone()
+    p2, s2 = wd.kv_pages.clone(), wd.kv_scale.clone()
+    mla.append_kv(c_new.to(DEV), k_new.to(DEV), p1, s1, wd.page_table, wd.ctx_lens)
+    mla.append_kv(c_new.to(DEV), k_new.to(DEV), p2, s2, wide[:, :n], wd.ctx_lens)
+    torch.cuda.synchronize()
+    assert torch.equal(p1, p2) and torch.equal(s1, s2)
+
+
 def test_append_host_errors():
     w = W.make_workload("single_query_256").to(DEV)
     c_new, k_new = _fresh_rows(1, 1, 61)

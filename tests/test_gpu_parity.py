@@ -80,6 +80,23 @@ def test_page_relabelling_is_bit_identical(kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+def test_padded_page_table_rows_are_bit_identical(kernel):
+    """A page table whose rows are the first columns of a wider array (row
+    stride larger than the row): the same pages, the same bits."""
+    w = W.make_workload("spec_verify_small", B=3, kv=W.KV_FP8, ctx_override=("uniform", 200, 900))
+    a = _run(w, kernel)
+    B, n = w.page_table.shape
+    wide = torch.full((B, n + 37), -1, dtype=torch.int32)
+    wide[:, :n] = w.page_table
+    wd = w.to(DEV)
+    pt = wide.to(DEV)[:, :n]
+    assert pt.stride(0) == n + 37 and not pt.is_contiguous()
+    b = mla.decode(wd.q_lat, wd.q_pe, wd.kv_pages, wd.kv_scale, pt, wd.ctx_lens, wd.sm_scale, kernel=kernel)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 def test_head_padding_is_bit_identical(kernel):
     w = W.make_workload("spec_verify_small", B=3, ctx_override=("uniform", 200, 900))
     o12, l12 = _run(w, kernel)
