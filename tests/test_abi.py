@@ -180,3 +180,20 @@ def test_binding_argument_counts_match_prototypes(lib):
         fn = getattr(lib, name)
         assert fn.argtypes is not None, f"{name}: the binding sets no argtypes"
         assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def test_valid_calls_without_a_gpu_fail_with_a_cuda_status(lib):
+    """With no CUDA device, well-formed calls return MLA_ERR_CUDA and record
+    the CUDA error; nothing crashes and nothing falls back to the CPU.  (Only
+    where no device exists: these calls pass host buffers.)"""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    buf = ctypes.create_string_buffer(1 << 16)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) & ~255)
+    d = _dims()
+    assert lib.mla_decode_workspace_size(ctypes.byref(d)) == -4
+    assert lib.mla_decode(p, p, p, None, p, p, 0.1, p, p, ctypes.byref(d), p, 4096, None) == -4
+    assert lib.mla_last_cuda_error() != 0
+    assert lib.mla_merge_partials(p, p, 2, 4, p, 0, p, None) == -4
+    assert lib.mla_append_kv(p, p, p, None, p, p, ctypes.byref(d), None, None) == -4
