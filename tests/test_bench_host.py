@@ -8,7 +8,6 @@ import shutil
 import subprocess
 import sys
 
-import pytest
 
 import bench
 import mla_workloads as W
