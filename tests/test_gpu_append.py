@@ -124,7 +124,8 @@ def test_append_through_padded_page_table():
     mla.append_kv(c_new.to(DEV), k_new.to(DEV), p1, s1, wd.page_table, wd.ctx_lens)
     mla.append_kv(c_new.to(DEV), k_new.to(DEV), p2, s2, wide[:, :n], wd.ctx_lens)
     torch.cuda.synchronize()
-    assert torch.equal(p1, p2) and torch.equal(s1, s2)
+    # bit patterns: unused slots hold NaN scales, which compare unequal as floats
+    assert torch.equal(p1, p2) and torch.equal(s1.view(torch.int32), s2.view(torch.int32))
 
 
 def test_append_host_errors():
