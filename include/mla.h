@@ -165,10 +165,10 @@ MLA_API int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages
 
 /*
  * mla_decode without a caller-provided workspace, for callers that cannot
- * allocate device memory when they decode (for example while a CUDA graph is
- * captured in a mode that forbids allocation, or inside a runtime whose device
- * memory all belongs to another allocator).  The pages describe no such
- * entry point; it is a service of this library, not part of the method.
+ * allocate device memory when they decode (for example a runtime whose device
+ * memory all belongs to another allocator, or a plugin that must not grow the
+ * process's device footprint per call).  The pages describe no such entry
+ * point; it is a service of this library, not part of the method.
  *
  * Same arguments and results as mla_decode, minus the workspace.  The scratch
  * is one fixed 32 MiB array in device memory, defined in the library, held by
@@ -178,7 +178,11 @@ MLA_API int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages
  *     MLA_ERR_WORKSPACE and launches nothing.
  *   - The first call on each device looks up the array's device address (a
  *     host-side runtime query, made with that device current).  Make that
- *     first call before any stream capture on the device.
+ *     first call before any stream capture on the device.  The address is
+ *     kept for the life of the process: after cudaDeviceReset (or any loss of
+ *     the device's primary context) this entry point must not be called again.
+ *   - Argument errors are reported before anything is enqueued, as for
+ *     mla_decode.
  *   - Each call clears the array's error word on `stream`, then runs the
  *     decode there.  The device error word is not reported.
  *   - All calls share the one array, so calls that can overlap on the GPU

@@ -48,6 +48,8 @@ int check_dims(const mla_dims *d) {
     if ((int64_t)d->B * d->T * d->H > ((int64_t)1 << 29) - 1) return MLA_ERR_INVALID_ARG;  // merge grid
     if (d->num_pages < 1 || d->max_pages_per_seq < 1 || d->page_table_stride < d->max_pages_per_seq)
         return MLA_ERR_INVALID_ARG;
+    // the device schedule sums page counts of all sequences in 32-bit integers
+    if ((int64_t)d->B * d->max_pages_per_seq > (int64_t)INT32_MAX) return MLA_ERR_INVALID_ARG;
     if (d->kv_dtype != MLA_KV_BF16 && d->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
     if (d->kv_scale_per_tensor != 0 && d->kv_scale_per_tensor != 1) return MLA_ERR_INVALID_ARG;
     if (d->kv_scale_per_tensor && d->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
@@ -91,6 +93,22 @@ int make_plan(const mla_dims *d, Plan *pl) {
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Checks of mla_decode's arguments that need no CUDA call (the workspace aside).
+int check_decode_args(const void *q_lat, const void *q_pe, const void *kv_pages, const float *kv_scale,
+                      const int32_t *page_table, const int32_t *ctx_lens, float sm_scale, const void *out,
+                      const float *lse, const mla_dims *dims) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!q_lat || !q_pe || !kv_pages || !page_table || !ctx_lens || !out) return MLA_ERR_INVALID_ARG;
+    if ((dims->kv_dtype == MLA_KV_FP8_E4M3) != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q_lat, 16) || !aligned(q_pe, 16) || !aligned(kv_pages, 16) || !aligned(out, 16) ||
+        !aligned(page_table, 4) || !aligned(ctx_lens, 4) || (kv_scale && !aligned(kv_scale, 16)) ||
+        (lse && !aligned(lse, 4)))
+        return MLA_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || sm_scale == INFINITY || sm_scale == -INFINITY) return MLA_ERR_INVALID_ARG;
+    return MLA_OK;
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -108,15 +126,8 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
                const int32_t *page_table, const int32_t *ctx_lens, float sm_scale, void *out,
                float *lse, const mla_dims *dims, void *workspace, size_t workspace_bytes,
                mla_stream_t stream) {
-    int rc = check_dims(dims);
+    int rc = check_decode_args(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, out, lse, dims);
     if (rc) return rc;
-    if (!q_lat || !q_pe || !kv_pages || !page_table || !ctx_lens || !out) return MLA_ERR_INVALID_ARG;
-    if ((dims->kv_dtype == MLA_KV_FP8_E4M3) != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
-    if (!aligned(q_lat, 16) || !aligned(q_pe, 16) || !aligned(kv_pages, 16) || !aligned(out, 16) ||
-        !aligned(page_table, 4) || !aligned(ctx_lens, 4) || (kv_scale && !aligned(kv_scale, 16)) ||
-        (lse && !aligned(lse, 4)))
-        return MLA_ERR_INVALID_ARG;
-    if (!(sm_scale == sm_scale) || sm_scale == INFINITY || sm_scale == -INFINITY) return MLA_ERR_INVALID_ARG;
     if (!workspace || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
     Plan pl;
     rc = make_plan(dims, &pl);
@@ -178,13 +189,11 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
 // Allocation-free decode.
 //
 // Some callers cannot call cudaMalloc (or any allocating routine) at the point
-// where they decode: code running while a CUDA graph is being captured in a
-// mode that forbids allocation, runtimes whose device memory is entirely
-// owned by another allocator arena, or plugins that must not grow the
-// process's device footprint per call.  For them the library keeps one fixed
-// scratch array in device memory (every GPU that loads the library holds it
-// until the process exits) and runs the ordinary decode with that array as
-// its workspace.
+// where they decode: runtimes whose device memory is entirely owned by another
+// allocator arena, or plugins that must not grow the process's device
+// footprint per call.  For them the library keeps one fixed scratch array in
+// device memory (every GPU that loads the library holds it until the process
+// exits) and runs the ordinary decode with that array as its workspace.
 // ---------------------------------------------------------------------------
 static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -194,7 +203,9 @@ static std::mutex g_noalloc_mu;
 
 // Device address of the scratch array on the current device.  The host-side
 // symbol is only a stand-in: the address must come from the runtime, once per
-// device, with that device current.
+// device, with that device current.  The address is kept for the life of the
+// process, so it does not survive a reset of the device (cudaDeviceReset) or
+// a re-created primary context.
 static int noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -220,7 +231,8 @@ static int noalloc_scratch(void **out) {
 int mla_decode_noalloc(const void *q_lat, const void *q_pe, const void *kv_pages, const float *kv_scale,
                        const int32_t *page_table, const int32_t *ctx_lens, float sm_scale, void *out,
                        float *lse, const mla_dims *dims, mla_stream_t stream) {
-    int rc = check_dims(dims);
+    // every check that can fail without a CUDA call comes before anything is enqueued
+    int rc = check_decode_args(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, out, lse, dims);
     if (rc) return rc;
     const int64_t need = mla_decode_workspace_size(dims);
     if (need < 0) return (int)need;

@@ -60,7 +60,9 @@ BAD_DIMS = [dict(B=0), dict(T=0), dict(T=9), dict(H=0), dict(T=8, H=129), dict(n
             dict(max_pages_per_seq=0), dict(page_table_stride=8), dict(kv_dtype=2),
             dict(out_dtype=5), dict(num_splits=-1), dict(kernel=7),
             dict(B=1 << 26, T=8, H=1),                 # 2^29 query rows: past the merge grid
-            dict(kv_scale_per_tensor=2), dict(kv_scale_per_tensor=1)]  # the latter with a bf16 cache
+            dict(kv_scale_per_tensor=2), dict(kv_scale_per_tensor=1),  # the latter with a bf16 cache
+            # B * max_pages_per_seq = 2^32 page slots: past the device schedule's 32-bit sums
+            dict(B=1 << 20, max_pages_per_seq=1 << 12, page_table_stride=1 << 12)]
 
 
 @pytest.mark.parametrize("bad", BAD_DIMS, ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))
@@ -91,6 +93,22 @@ def test_null_pointers_rejected_without_gpu(lib):
     # workspace missing or misaligned
     assert lib.mla_decode(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), None, 4096, None) == -3
     assert lib.mla_decode(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), q, 4096, None) == -3
+
+
+def test_noalloc_argument_errors_enqueue_nothing(lib):
+    """mla_decode_noalloc reports argument errors before it touches the
+    device: without a GPU a call that reached its first CUDA call would
+    return MLA_ERR_CUDA (-4), not MLA_ERR_INVALID_ARG (-1)."""
+    d = _dims()
+    buf = ctypes.create_string_buffer(4096 + 256)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 255) & ~255)
+    q = ctypes.c_void_p(p.value + 8)
+    assert lib.mla_decode_noalloc(None, p, p, None, p, p, 0.1, p, None, ctypes.byref(d), None) == -1
+    assert lib.mla_decode_noalloc(p, p, q, None, p, p, 0.1, p, None, ctypes.byref(d), None) == -1
+    assert lib.mla_decode_noalloc(p, p, p, p, p, p, 0.1, p, None, ctypes.byref(d), None) == -1
+    assert lib.mla_decode_noalloc(p, p, p, None, p, p, float("inf"), p, None, ctypes.byref(d), None) == -1
+    bad = _dims(T=0)
+    assert lib.mla_decode_noalloc(p, p, p, None, p, p, 0.1, p, None, ctypes.byref(bad), None) == -1
 
 
 def test_merge_argument_checks_without_gpu(lib):

@@ -1,14 +1,18 @@
 """The allocation-free decode entry point, checked against the ordinary one.
 
 ``mla_decode_noalloc`` is for callers that cannot allocate device memory at
-the point where they decode -- a CUDA graph captured in a mode that forbids
-allocation, or a runtime whose device memory all belongs to another
-allocator.  It runs the same kernels as ``mla_decode`` with a fixed scratch
-array defined inside the library instead of a caller-provided workspace.
+the point where they decode -- a runtime whose device memory all belongs to
+another allocator, or a plugin that must not grow the process's device
+footprint per call.  It runs the same kernels as ``mla_decode`` with a fixed
+scratch array defined inside the library instead of a caller-provided
+workspace.
 
 Each case calls it twice in a row, through the C ABI, and compares both
-results with ``mla_decode`` on the same inputs, within the parity tolerance
-used elsewhere in the suite.  This file is named to be collected last, so
+results with ``mla_decode`` on the same inputs: within the parity tolerance
+used elsewhere in the suite, and bit for bit, since both entry points run
+the same deterministic kernels (a stale value left in the shared scratch
+array would show up as a difference).  The device's free memory must not
+change across the second call.  This file is named to be collected last, so
 that a run stopping at the first failure has run everything else first.
 """
 import ctypes
@@ -44,16 +48,24 @@ def test_noalloc_matches_decode_twice(name, kw):
     ref_o, ref_l = mla.decode_workload(w)
     torch.cuda.synchronize()
     tol = out_rel_tol(w.kv_dtype) * ref_o.float().abs().max().item() + 1e-3
-    for _ in range(2):
-        out = torch.full_like(ref_o, float("nan"))
-        lse = torch.full_like(ref_l, float("nan"))
-        assert _noalloc(w, out, lse) == 0
+    outs = [torch.full_like(ref_o, float("nan")) for _ in range(2)]
+    lses = [torch.full_like(ref_l, float("nan")) for _ in range(2)]
+    free_before = None
+    for i in range(2):
+        if i == 1:
+            torch.cuda.synchronize()
+            free_before = torch.cuda.mem_get_info()[0]
+        assert _noalloc(w, outs[i], lses[i]) == 0
         torch.cuda.synchronize()
+        if i == 1:
+            assert torch.cuda.mem_get_info()[0] == free_before
+        out, lse = outs[i], lses[i]
         assert torch.isfinite(out.float()).all()
         assert (out.float() - ref_o.float()).abs().max().item() <= tol
         fin = torch.isfinite(ref_l)
         assert torch.equal(fin, torch.isfinite(lse))
         assert (lse[fin] - ref_l[fin]).abs().max().item() <= LSE_TOL
+        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
 
 
 def test_noalloc_rejects_work_beyond_its_scratch():
