@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-append", dest="append", action="store_false",
                     help="skip timing the cache writer (mla_append_kv) on the workload's new tokens")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip timing every workload of the problem statement after the headline one")
     return ap.parse_args()
 
 
@@ -346,6 +348,246 @@ def time_append(mla, w, kv, sc, L, stream, reps=50):
             "note": "one launch per layer, timed apart from the decode step"}
 
 
+class LayerStack:
+    """One decode step of an L-layer MLA stack: L calls of the library over L
+    separate copies of a workload's paged cache (same contents, own memory),
+    for the same query rows.  A context-partitioned workload decodes its
+    partitions to fp32 partials and merges them with mla_merge_partials."""
+
+    def __init__(self, mla, w, L, dev, args, parts=None):
+        self.mla, self.w, self.L, self.args = mla, w, L, args
+        self.units = [parts] if parts else [[w]]
+        srcs = parts if parts else [w]
+        self.kv = [[s.kv_pages if i == 0 else s.kv_pages.clone() for s in srcs] for i in range(L)]
+        self.sc = [[None if s.kv_scale is None else (s.kv_scale if i == 0 else s.kv_scale.clone())
+                    for s in srcs] for i in range(L)]
+        self.srcs = srcs
+        B, T, H = w.B, w.T, w.H
+        self.q_lat = torch.stack([w.q_lat] * L)
+        self.q_pe = torch.stack([w.q_pe] * L)
+        self.outs = torch.empty((L, B, T, H, 512), dtype=torch.bfloat16, device=dev)
+        self.lses = torch.empty((L, B, T, H), dtype=torch.float32, device=dev)
+        self.part_out = self.part_lse = None
+        if parts:
+            self.part_out = torch.empty((L, len(parts), B, T, H, 512), dtype=torch.float32, device=dev)
+            self.part_lse = torch.empty((L, len(parts), B, T, H), dtype=torch.float32, device=dev)
+        need = 0
+        self.calls_per_layer = 0
+        for s in srcs:
+            d = mla.make_dims(w.q_lat, s.kv_pages, s.page_table, kernel=args.kernel,
+                              num_splits=args.num_splits, vis_lens=s.vis_lens,
+                              out_dtype=torch.float32 if parts else torch.bfloat16, kv_scale=s.kv_scale)
+            n = mla.workspace_size(d)
+            need = max(need, n)
+            self.calls_per_layer += 2 if n > 256 else 1
+        if parts:
+            self.calls_per_layer += 1
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        n_dec = len(srcs)
+        self.ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+                    for _ in range(n_dec + (1 if parts else 0))] for _ in range(L)]
+        for e in (x for a in self.ev for b in a for x in b):
+            e.record()      # torch creates CUDA events lazily: make the handles exist
+
+    def layer(self, i, events=False):
+        mla, parts = self.mla, self.part_out is not None
+        for k, s in enumerate(self.srcs):
+            e = self.ev[i][k]
+            if events:
+                e[0].record()
+            out = self.part_out[i, k] if parts else self.outs[i]
+            lse = self.part_lse[i, k] if parts else self.lses[i]
+            mla.decode(self.q_lat[i], self.q_pe[i], self.kv[i][k], self.sc[i][k], s.page_table, s.ctx_lens,
+                       s.sm_scale, out=out, lse=lse, vis_lens=s.vis_lens, kernel=self.args.kernel,
+                       num_splits=self.args.num_splits, workspace=self.ws,
+                       stage_event=e[1] if events else None)
+            if events:
+                e[2].record()
+        if parts:
+            e = self.ev[i][-1]
+            if events:
+                e[0].record()
+                e[1].record()
+            mla.merge_partials(self.part_out[i], self.part_lse[i], out=self.outs[i], lse=self.lses[i])
+            if events:
+                e[2].record()
+
+    def step(self, events=False):
+        for i in range(self.L):
+            self.layer(i, events)
+
+    def split_us(self):
+        """(attention, merge) device microseconds of the last replay, per layer."""
+        att = mer = 0.0
+        for i in range(self.L):
+            for e in self.ev[i]:
+                att += event_ms(e[0], e[1]) * 1e3
+                mer += event_ms(e[1], e[2]) * 1e3
+        return att / self.L, mer / self.L
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    return g
+
+
+def time_replays(graph, steps):
+    """Device seconds of ``steps`` back-to-back replays (CUDA events on the
+    stream the replays are launched on)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / 1e3
+
+
+def kernel_split(stack, graph_ev, rounds=6, burst=4):
+    """Attention and merge microseconds per layer from the event-instrumented
+    graph, replayed ``burst`` times back to back (no host synchronisation in
+    between, so the GPU stays busy as in the timed loop) and read after the
+    last replay of each round."""
+    att, mer = [], []
+    for _ in range(rounds):
+        for _ in range(burst):
+            graph_ev.replay()
+        torch.cuda.synchronize()
+        a, m = stack.split_us()
+        att.append(a)
+        mer.append(m)
+    att.sort()
+    mer.sort()
+    return att[len(att) // 2], mer[len(mer) // 2]
+
+
+def roof_fraction(units_layer, us, peaks, bound):
+    """Achieved rate of one layer against the roofline that binds it."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    e4m3 = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    gbs = units_layer["total_bytes"] / us / 1e3
+    tfs = units_layer["flops"] / us / 1e6
+    if bound == "hbm":
+        return {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+    return {"bound": "tensor (e4m3)", "achieved": tfs, "peak": e4m3, "unit": "TFLOP/s", "frac": tfs / e4m3,
+            "note": "algorithmic flop; the exact hi/lo operand split issues twice as many e4m3 MMAs"}
+
+
+# Binding roofline per workload (flop per cached byte against the B200 ridge):
+# one or a few query rows per sequence are HBM-bound, 288 rows per sequence
+# (B x 3 drafts x 96 heads) are tensor-bound.
+BINDING = {"single_query_256": "hbm", "spec_verify_small": "hbm", "batched_verify_fp8_32k": "tensor",
+           "long_ctx_142k": "hbm", "ragged_dcp8": "tensor"}
+PER_CONFIG = [("single_query_256", None), ("spec_verify_small", None), ("batched_verify_fp8_32k", None),
+              ("long_ctx_142k", None), ("long_ctx_142k", W.KV_BF16), ("ragged_dcp8", None)]
+
+
+def measure_config(mla, name, kv, dev, args, peaks, stream, seconds=0.4):
+    """Every workload of the problem statement at full size, timed like the
+    headline: a graph of L layers over L cache copies (L chosen so one step
+    reads at least 1 GB of KV, above the 126 MB L2); a workload too small for
+    that (the 256-position sanity case) flushes L2 before each step and is
+    timed step by step."""
+    w = W.make_workload(name, device=dev, kv=kv)
+    parts = W.partition_round_robin(w, W.CONFIGS[name].partitions) if W.CONFIGS[name].partitions > 1 else None
+    u1 = step_units(w, 1)
+    L = max(1, min(24, -(-int(1e9) // max(1, u1["kv_bytes"]))))
+    flush = L * u1["kv_bytes"] < 4 * 126e6
+    stack = LayerStack(mla, w, L, dev, args, parts)
+    stack.step()
+    torch.cuda.synchronize()
+    g = capture(stack.step, stream)
+    g_ev = capture(lambda: stack.step(True), stream)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    if flush:
+        scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        times = []
+        for _ in range(20):
+            scratch.fill_(1)
+            times.append(time_replays(g, 1))
+        times.sort()
+        step_s = times[len(times) // 2]
+        steps = 20
+        del scratch
+    else:
+        t1 = time_replays(g, 1)
+        steps = max(3, min(2000, int(seconds / max(t1, 1e-6))))
+        step_s = time_replays(g, steps) / steps
+    att, mer = kernel_split(stack, g_ev)
+    layer_us = step_s / L * 1e6
+    res = {"kv": w.kv_label(), "B": w.B, "T": w.T, "H": w.H, "layers": L, "steps": steps,
+           "l2": "flushed before each step" if flush else f"{L * u1['kv_bytes'] / 1e9:.2f} GB of KV per step",
+           "layer_us": layer_us, "attention_us": att, "merge_us": mer,
+           "split_within_step": att + mer <= layer_us * 1.05,
+           "kv_read_gbs": u1["kv_bytes"] / layer_us / 1e3,
+           "seq_steps_per_s": w.B / (layer_us * 1e-6),
+           "hbm_fraction_of_8TBs": u1["kv_bytes"] / layer_us / 1e3 / NOMINAL_HBM_GBS}
+    if parts:
+        res["partitions"] = len(parts)
+    res["roof"] = roof_fraction(u1, layer_us, peaks, BINDING[name])
+    res["roof_attention_kernel"] = roof_fraction(u1, att, peaks, BINDING[name]) if not parts else None
+    del g, g_ev, stack
+    torch.cuda.empty_cache()
+    return res
+
+
+def e2e_overlapped(stack, steps, world, dev):
+    """The same step through the public API with the query rows coming from
+    pinned host memory and the outputs going back to it every step.  The two
+    copy directions run on streams of their own, ordered with the kernels by
+    per-layer events: layer i's inputs for the next step are copied once its
+    decode has read them, its outputs once it has written them."""
+    L = stack.L
+    h_qlat = torch.empty(stack.q_lat.shape, dtype=stack.q_lat.dtype, pin_memory=True).copy_(stack.q_lat)
+    h_qpe = torch.empty(stack.q_pe.shape, dtype=stack.q_pe.dtype, pin_memory=True).copy_(stack.q_pe)
+    h_out = torch.empty(stack.outs.shape, dtype=stack.outs.dtype, pin_memory=True)
+    h_lse = torch.empty(stack.lses.shape, dtype=stack.lses.dtype, pin_memory=True)
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(L)]
+    ev_done = [torch.cuda.Event() for _ in range(L)]
+    ev_saved = [torch.cuda.Event() for _ in range(L)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for s in range(steps):
+        with torch.cuda.stream(up):
+            for i in range(L):
+                if s > 0:
+                    up.wait_event(ev_done[i])       # the previous step's decode of layer i has read q[i]
+                stack.q_lat[i].copy_(h_qlat[i], non_blocking=True)
+                stack.q_pe[i].copy_(h_qpe[i], non_blocking=True)
+                ev_in[i].record(up)
+        for i in range(L):
+            comp.wait_event(ev_in[i])
+            if s > 0:
+                comp.wait_event(ev_saved[i])        # the previous step's out[i] is on the host
+            stack.layer(i)
+            ev_done[i].record(comp)
+        with torch.cuda.stream(down):
+            for i in range(L):
+                down.wait_event(ev_done[i])
+                h_out[i].copy_(stack.outs[i], non_blocking=True)
+                h_lse[i].copy_(stack.lses[i], non_blocking=True)
+                ev_saved[i].record(down)
+    comp.wait_stream(down)
+    comp.wait_stream(up)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3
+    h2d = h_qlat.numel() * h_qlat.element_size() + h_qpe.numel() * h_qpe.element_size()
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+    return t, h2d, d2h
+
+
 def run_ours(args, rank, world, local_rank):
     import mla_latent_attention_b200 as mla
     dev = torch.device("cuda", local_rank)
@@ -353,59 +595,20 @@ def run_ours(args, rank, world, local_rank):
     w = make_bench_workload(args, device=dev)
     L = args.layers
     units = step_units(w, L)
-    # each layer: its own copy of the paged cache (same contents, own memory)
-    kv = [w.kv_pages] + [w.kv_pages.clone() for _ in range(L - 1)]
-    sc = None if w.kv_scale is None else [w.kv_scale] + [w.kv_scale.clone() for _ in range(L - 1)]
-    B, T, H = w.B, w.T, w.H
-    q_lat = torch.stack([w.q_lat] * L)          # [L,B,T,H,512]
-    q_pe = torch.stack([w.q_pe] * L)
-    outs = torch.empty((L, B, T, H, 512), dtype=torch.bfloat16, device=dev)
-    lses = torch.empty((L, B, T, H), dtype=torch.float32, device=dev)
-    dims = mla.make_dims(w.q_lat, w.kv_pages, w.page_table, kernel=args.kernel,
-                         num_splits=args.num_splits)
-    ws_bytes = mla.workspace_size(dims)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    launches_per_call = 2 if ws_bytes > 256 else 1
-    ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
-    ev_m = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
-    ev_b = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
-
-    def one_step(timed_events):
-        for i in range(L):
-            if timed_events:
-                ev_a[i].record()
-            mla.decode(q_lat[i], q_pe[i], kv[i], None if sc is None else sc[i], w.page_table,
-                       w.ctx_lens, w.sm_scale, out=outs[i], lse=lses[i], kernel=args.kernel,
-                       num_splits=args.num_splits, workspace=ws,
-                       stage_event=ev_m[i] if timed_events else None)
-            if timed_events:
-                ev_b[i].record()
-
-    # torch creates CUDA events lazily: record each once so its handle exists
-    # before it is handed to the library or captured
-    for e in ev_a + ev_m + ev_b:
-        e.record()
-    # eager warm-up (sets kernel attributes), then capture one step as a graph;
+    stack = LayerStack(mla, w, L, dev, args)
+    launches_per_call = stack.calls_per_layer
+    # eager warm-up (sets kernel attributes), then one step captured as a graph;
     # a second graph of the same step carries per-layer event nodes, for the
     # per-kernel durations only (event nodes are kept out of the timed graph)
-    one_step(False)
+    stack.step()
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
-    graph = torch.cuda.CUDAGraph()
-    graph_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(graph, stream=stream):
-            one_step(False)
-        with torch.cuda.graph(graph_ev, stream=stream):
-            one_step(True)
-    torch.cuda.synchronize()
+    graph = capture(stack.step, stream)
+    graph_ev = capture(lambda: stack.step(True), stream)
     for _ in range(max(3, args.warmup)):
         graph.replay()
     torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    graph.replay()
-    torch.cuda.synchronize()
-    est = time.perf_counter() - t0
+    est = time_replays(graph, 1)
     steps = args.steps if args.steps is not None else max(10, min(20000, int(3.0 / max(est, 1e-6))))
 
     sampler = ClockSampler(local_rank)
@@ -416,70 +619,47 @@ def run_ours(args, rank, world, local_rank):
         graph.replay()
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(steps):
-        graph.replay()
-    stop.record()
-    torch.cuda.synchronize()
+    elapsed = time_replays(graph, steps)
     if world > 1:
         torch.distributed.barrier()
-    elapsed = start.elapsed_time(stop) / 1e3
-    # per-kernel durations: steps of the graph with event nodes, read one by one
-    dec, mer = [], []
-    for _ in range(12):
-        graph_ev.replay()
-        torch.cuda.synchronize()
-        dec += [event_ms(ev_a[i], ev_m[i]) / 1e3 for i in range(L)]
-        mer += [event_ms(ev_m[i], ev_b[i]) / 1e3 for i in range(L)]
-    clocks = sampler.stop()
-
+    dec_us, mer_us = kernel_split(stack, graph_ev)
     max_elapsed = max_over_ranks(elapsed, world, dev)
 
-    # end to end through the public API with host buffers: per step the query
-    # rows of every layer go host->device and the outputs come back.
-    h_qlat = torch.empty(q_lat.shape, dtype=q_lat.dtype, pin_memory=True).copy_(q_lat)
-    h_qpe = torch.empty(q_pe.shape, dtype=q_pe.dtype, pin_memory=True).copy_(q_pe)
-    h_out = torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True)
-    h_lse = torch.empty(lses.shape, dtype=lses.dtype, pin_memory=True)
     e2e_steps = max(3, min(steps, 200))
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        q_lat.copy_(h_qlat, non_blocking=True)
-        q_pe.copy_(h_qpe, non_blocking=True)
-        one_step(False)
-        h_out.copy_(outs, non_blocking=True)
-        h_lse.copy_(lses, non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_time = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    e2e_time, h2d, d2h = e2e_overlapped(stack, e2e_steps, world, dev)
+    e2e_time = max_over_ranks(e2e_time, world, dev)
     e2e_value = world * e2e_steps * units["kv_bytes"] / e2e_time / 1e9
-    h2d = (h_qlat.numel() * h_qlat.element_size() + h_qpe.numel() * h_qpe.element_size())
-    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
 
     # after every decode measurement: the writer changes the caches' last T slots
-    append = time_append(mla, w, kv, sc, L, stream) if args.append else None
+    kv0 = [k[0] for k in stack.kv]
+    sc0 = [c[0] for c in stack.sc]
+    append = time_append(mla, w, kv0, None if sc0[0] is None else sc0, L, stream) if args.append else None
+
+    peaks, peak_src = load_peaks()
+    per_config = None
+    if args.per_config and world == 1:
+        del graph, graph_ev
+        per_config = {}
+        for name, kv in PER_CONFIG:
+            key = name if kv is None else f"{name}:{kv}"
+            per_config[key] = measure_config(mla, name, kv, dev, args, peaks, stream)
+    clocks = sampler.stop()
 
     if rank != 0:
         return
-    peaks, peak_src = load_peaks()
     value = world * steps * units["kv_bytes"] / max_elapsed / 1e9
-    dec_avg = sum(dec) / len(dec)
+    layer_us = max_elapsed / steps / L * 1e6
     per_launch_bytes = units["total_bytes"] / L
     per_launch_flops = units["flops"] / L
-    achieved_gbs = per_launch_bytes / dec_avg / 1e9
+    achieved_gbs = per_launch_bytes / dec_us / 1e3
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved_gbs / hbm_peak, "traffic": recorded_traffic(args.workload, w.kv_label()),
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "kernel": "mla decode attention kernel", "peak_source": f"{peak_src} hbm_gbs",
-                "avg_launch_us": dec_avg * 1e6, "merge_avg_launch_us": sum(mer) / len(mer) * 1e6}
-    tflops = per_launch_flops / dec_avg / 1e12
+                "avg_launch_us": dec_us, "merge_avg_launch_us": mer_us, "layer_us": layer_us,
+                "split_within_step": dec_us + mer_us <= layer_us * 1.05}
+    tflops = per_launch_flops / dec_us / 1e6
     kernel_dtype = {"simt": "f32"}.get(args.kernel, "e4m3" if w.kv_dtype == W.KV_FP8 else "bf16")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
@@ -492,19 +672,22 @@ def run_ours(args, rank, world, local_rank):
         "tensor_tflops": tflops,
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "note": "host copies on two side streams, overlapped with other layers' kernels"},
         "gpu_launches": steps * L * launches_per_call,
         "clocks": clocks,
     }
     if append is not None:
         line["append"] = append
+    if per_config is not None:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
         st, rows, spent, threads = oracle_sample(w, L, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": units["kv_bytes"] / st / 1e9, "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": f"{rows} whole query rows of one layer ({spent:.1f} s), extrapolated to "
-                      f"{L} layers x {B * T * H} rows"}
+                      f"{L} layers x {w.B * w.T * w.H} rows"}
     print(json.dumps(line), flush=True)
 
 

@@ -114,6 +114,14 @@ typedef struct mla_dims {
                                      position; 1 = kv_scale points to ONE fp32 scale for the
                                      whole cache (a static, calibrated scale: "Kimi K2.6 DFlash
                                      on 8x MI300X", next steps) */
+    int32_t wait_limit_kcycles;   /* 0 = default: an on-chip wait of the tensor-core kernel
+                                     (for a copy, an MMA or another warp) gives up after about
+                                     4e9 SM cycles (about 2 s).  > 0: after this many thousand
+                                     cycles instead, for a tighter watchdog or to exercise the
+                                     stop.  A CTA whose wait gives up records MLA_DEV_TIMEOUT,
+                                     lets its copies and MMAs in flight finish, frees its tensor
+                                     memory and exits; its rows' results are unspecified.
+                                     Must be >= 0. */
 } mla_dims;
 
 /*

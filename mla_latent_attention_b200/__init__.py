@@ -28,7 +28,8 @@ MLA_OK = 0
 KV_BF16, KV_FP8 = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 KERNELS = {"auto": 0, "simt": 1, "tcgen05": 2}
-DEV_ERRORS = {0: "ok", 1: "bad page index", 2: "bad context length", 3: "bad visible count"}
+DEV_ERRORS = {0: "ok", 1: "bad page index", 2: "bad context length", 3: "bad visible count",
+              4: "an on-chip wait gave up"}
 EXPORTED = ("mla_decode_workspace_size", "mla_decode", "mla_decode_noalloc", "mla_merge_partials", "mla_append_kv",
             "mla_read_device_error", "mla_reset_device_error", "mla_status_string",
             "mla_last_cuda_error")
@@ -44,7 +45,8 @@ class Dims(ctypes.Structure):
                 ("page_table_stride", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
                 ("out_dtype", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("kernel", ctypes.c_int32), ("vis_lens", ctypes.c_void_p),
-                ("stage_event", ctypes.c_void_p), ("kv_scale_per_tensor", ctypes.c_int32)]
+                ("stage_event", ctypes.c_void_p), ("kv_scale_per_tensor", ctypes.c_int32),
+                ("wait_limit_kcycles", ctypes.c_int32)]
 
 
 def library_path() -> str:
@@ -115,7 +117,7 @@ def _kv_code(kv_pages):
 
 
 def make_dims(q_lat, kv_pages, page_table, *, out_dtype=torch.bfloat16, num_splits=0,
-              kernel="auto", vis_lens=None, stage_event=None, kv_scale=None) -> Dims:
+              kernel="auto", vis_lens=None, stage_event=None, kv_scale=None, wait_limit_kcycles=0) -> Dims:
     B, T, H = int(q_lat.shape[0]), int(q_lat.shape[1]), int(q_lat.shape[2])
     return Dims(B=B, T=T, H=H, num_pages=int(kv_pages.shape[0]),
                 max_pages_per_seq=int(page_table.shape[1]),
@@ -124,7 +126,8 @@ def make_dims(q_lat, kv_pages, page_table, *, out_dtype=torch.bfloat16, num_spli
                 num_splits=int(num_splits), kernel=KERNELS[kernel],
                 vis_lens=None if vis_lens is None else vis_lens.data_ptr(),
                 stage_event=None if stage_event is None else stage_event.cuda_event,
-                kv_scale_per_tensor=int(kv_scale is not None and kv_scale.numel() == 1))
+                kv_scale_per_tensor=int(kv_scale is not None and kv_scale.numel() == 1),
+                wait_limit_kcycles=int(wait_limit_kcycles))
 
 
 def workspace_size(dims: Dims) -> int:
@@ -149,13 +152,15 @@ def _need(t, name, dtype=None, device=None, shape=None):
 
 def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, out=None, lse=None,
            vis_lens=None, out_dtype=torch.bfloat16, num_splits=0, kernel="auto", workspace=None,
-           stream=None, stage_event=None):
+           stream=None, stage_event=None, wait_limit_kcycles=0):
     """Paged MLA decode (``mla_decode``).  Returns (out [B,T,H,512], lse [B,T,H] fp32).
 
     ``stage_event`` (a ``torch.cuda.Event``) is recorded between the attention
     kernel and the merge kernel, for timing the two apart.  A ``workspace``
     whose device error word will be read (``read_device_error``) must start
-    zeroed (``torch.zeros``, or ``reset_device_error`` once)."""
+    zeroed (``torch.zeros``, or ``reset_device_error`` once).
+    ``wait_limit_kcycles`` > 0 bounds every on-chip wait of the tensor-core
+    kernel to that many thousand SM cycles (``mla_dims.wait_limit_kcycles``)."""
     lib = load_library()
     dev = q_lat.device
     B, T, H = q_lat.shape[:3]
@@ -183,7 +188,8 @@ def decode(q_lat, q_pe, kv_pages, kv_scale, page_table, ctx_lens, sm_scale, *, o
     else:
         _need(lse, "lse", torch.float32, dev, (B, T, H))
     dims = make_dims(q_lat, kv_pages, page_table, out_dtype=out_dtype, num_splits=num_splits,
-                     kernel=kernel, vis_lens=vis_lens, stage_event=stage_event, kv_scale=kv_scale)
+                     kernel=kernel, vis_lens=vis_lens, stage_event=stage_event, kv_scale=kv_scale,
+                     wait_limit_kcycles=wait_limit_kcycles)
     need = workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)

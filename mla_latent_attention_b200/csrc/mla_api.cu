@@ -54,7 +54,7 @@ int check_dims(const mla_dims *d) {
     if (d->kv_scale_per_tensor != 0 && d->kv_scale_per_tensor != 1) return MLA_ERR_INVALID_ARG;
     if (d->kv_scale_per_tensor && d->kv_dtype != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
     if (d->out_dtype != MLA_OUT_BF16 && d->out_dtype != MLA_OUT_F32) return MLA_ERR_INVALID_ARG;
-    if (d->num_splits < 0) return MLA_ERR_INVALID_ARG;
+    if (d->num_splits < 0 || d->wait_limit_kcycles < 0) return MLA_ERR_INVALID_ARG;
     if (d->kernel != MLA_KERNEL_AUTO && d->kernel != MLA_KERNEL_SIMT && d->kernel != MLA_KERNEL_TCGEN05)
         return MLA_ERR_INVALID_ARG;
     return MLA_OK;
@@ -163,6 +163,7 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     p.n_groups = pl.n_groups;
     p.rows_per_group = pl.rows_per_group;
     p.sm_scale_log2 = sm_scale * kLog2e;
+    p.wait_limit = (uint64_t)dims->wait_limit_kcycles * 1000u;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     rc = pl.kernel == MLA_KERNEL_SIMT ? launch_simt(p, s) : launch_tc(p, s);

@@ -45,6 +45,7 @@ struct Problem {
     int n_groups;                 // row groups per sequence
     int rows_per_group;
     float sm_scale_log2;          // sm_scale * log2(e)
+    uint64_t wait_limit;          // SM cycles before an on-chip wait gives up; 0 = the kernel's default
 };
 
 __device__ __forceinline__ void report_error(int32_t *err, int code, int info) {

@@ -24,7 +24,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kQuarters = 4;
 constexpr int kFewParts = 16;
 constexpr int kBatch = 8;     // parts in flight per lane, one warp per unit
-constexpr int kCtaBatch = 8;  // the same, eight warps per unit
+constexpr int kCtaBatch = 10; // the same, eight warps per unit: 80 parts in one round of loads
 
 struct Online {
     float m = -INFINITY, s = 0.f;
@@ -169,6 +169,9 @@ __global__ void __launch_bounds__(kThreads, kCta ? 3 : 1) merge_internal_kernel(
     bool bad = false;
     pieces_of(p, b, &n_pieces, &piece_base, &bad);
     if (n_pieces < 2) return;  // finished by the decode kernel
+    // The kernel may start while the attention kernel is finishing (its
+    // schedule needs only ctx_lens); the partials are read after it is done.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // the pieces of row r are contiguous: [r][piece][512]
     const float *o0 = p.part_o + ((int64_t)r * p.max_pieces + piece_base) * kDl;
     const float *l0 = p.part_lse + (int64_t)r * p.max_pieces + piece_base;
@@ -206,11 +209,25 @@ int launch_merge_internal(const Problem &p, cudaStream_t stream) {
     // of pieces, only more slowly when there are many).
     const bool many = p.n_slots > 2 * p.B;
     const int64_t units = rows * kQuarters;
-    if (many)
-        merge_internal_kernel<true><<<(unsigned)units, kThreads, 0, stream>>>(p);
-    else
-        merge_internal_kernel<false><<<(unsigned)((units + kWarps - 1) / kWarps), kThreads, 0, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+    // a programmatic dependent of the attention kernel before it in the stream
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (many) {
+        cfg.gridDim = dim3((unsigned)units);
+        e = cudaLaunchKernelEx(&cfg, merge_internal_kernel<true>, p);
+    } else {
+        cfg.gridDim = dim3((unsigned)((units + kWarps - 1) / kWarps));
+        e = cudaLaunchKernelEx(&cfg, merge_internal_kernel<false>, p);
+    }
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         note_cuda_error(e);
         return MLA_ERR_CUDA;

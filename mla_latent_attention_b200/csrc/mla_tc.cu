@@ -40,8 +40,15 @@
 // than TAU (then O^T and the row sums are rescaled), and then to DELTA above
 // the new maximum, so after the first tile it rarely moves again.  Weights
 // are exp2(u - m2 + C), at most 2^(TAU+C), which keeps the e4m3 weights in
-// range.  Row sums are kept per lane and reduced once per piece.
-//
+// range.  Row sums are kept per lane and reduced once per piece.  The lanes
+// need not agree before they write a tile's weights: each warp writes them
+// with the current bound and flags the tile if one would exceed it; once
+// every warp has written the tile (the same barrier the value MMAs wait on),
+// a flagged tile takes a slow path in which all softmax warps agree on the
+// new bounds, rescale, and rewrite the weights, and the MMA warp issues that
+// tile's value MMAs only after the rewrite.  The first tile of every piece is
+// flagged (no bound yet); later ones almost never are.
+
 // Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA
 // records a timeout in the error word, stops, drains its outstanding copies
 // and MMAs and frees its tensor memory.
@@ -65,6 +72,11 @@ constexpr int kThreads = 64 + kSoftmaxThreads;      // warp 0 TMA, warp 1 MMA, w
 constexpr int kRpt = kN / kRowGroups;               // query rows per softmax thread
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 4000000000ull;  // SM cycles: about two seconds
+
+// The limit of every wait in the main work: the caller's (mla_dims), else
+// kWaitLimit.  The waits that drain a CTA's copies and MMAs before it exits
+// always keep kWaitLimit.
+__device__ __forceinline__ uint64_t wait_limit(const Problem &p) { return p.wait_limit ? p.wait_limit : kWaitLimit; }
 constexpr int kDevTimeout = 4;
 
 template <bool kFp8>
@@ -76,10 +88,21 @@ struct Cfg {
     static constexpr uint32_t kColS1 = 64;                                         // second S^T buffer
     static constexpr uint32_t kColO = 128;
     static constexpr uint32_t kOStride = kFp8 ? 96u : 64u;                         // O block m at kColO + m*stride
-    // KV stage: chunks of [128 positions][128 B]; FP8 adds the RoPE chunk [128][64 B]
-    static constexpr int kChunkBytes = kTileM * 128;                              // 16384
-    static constexpr int kVChunks = kFp8 ? 4 : 8;                                 // chunks holding c_kv
-    static constexpr int kStageBytes = kFp8 ? 4 * kChunkBytes + kTileM * 64 : 9 * kChunkBytes;
+    // KV stage.  The MMAs read the tile as 128-byte-wide column chunks (FP8: 4
+    // chunks of 128 latent dims; bf16: 9 chunks of 64 dims, the last one the
+    // RoPE part) of 128 positions, each chunk a stack of 8-position x 128 B
+    // swizzle atoms.  Byte offset of (8-position group g, chunk c):
+    //   g * kGroupStride + c * kChunkStride
+    // FP8: one 8 KB box per page lands [half][chunk][8 rows][128 B], so the
+    //   group stride is 4 KB and the chunks are 1 KB apart; the RoPE part is a
+    //   separate [128 positions][64 B] region at kRopeOff.
+    // bf16: one 2 KB box per (page, chunk): chunks of [128 positions][128 B].
+    static constexpr int kDimChunks = kFp8 ? 4 : 8;                               // 128-B chunks of c_kv
+    static constexpr int kGroupStride = kFp8 ? 4096 : 1024;
+    static constexpr int kChunkStride = kFp8 ? 1024 : kTileM * 128;
+    static constexpr int kRopeOff = kFp8 ? 4 * 16384 : 8 * kTileM * 128;
+    static constexpr int kStageBytes = kFp8 ? 4 * 16384 + kTileM * 64 : 9 * kTileM * 128;
+    static constexpr int kVChunks = kFp8 ? 1 : 8;                                 // parts holding c_kv
     static constexpr int kKvOff = 0;
     static constexpr int kScaleOff = kKvOff + kStages * kStageBytes;               // FP8: 512 B / stage
     static constexpr int kScaleBytes = kFp8 ? kTileM * 4 : 0;
@@ -94,13 +117,13 @@ struct Cfg {
     static constexpr int kPBytes = (kNMma / kPGroupRows) * kTileM * 16;           // 12288 both
     static constexpr int kPLoOff = kFp8 ? (kN / 16) * kTileM * 16 : 0;             // lo rows start (group 3)
     static constexpr int kMiscOff = kPOff + 2 * kPBytes;                           // P double-buffered
-    // Each stage is filled and freed in parts: the value chunks (FP8 4 x 128
-    // dims, bf16 8 x 64 dims) and the RoPE chunk, so the next tile's copies
-    // start as soon as the previous tile's MMAs are done with each part.
+    // Each stage is filled and freed in parts: the c_kv part (FP8: one part,
+    // with the per-position scales; bf16: 8 chunks of 64 dims) and the RoPE
+    // part, which the score MMAs alone read and so is freed first.
     static constexpr int kParts = kVChunks + 1;
     static constexpr int kRope = kVChunks;                                        // part index of the RoPE chunk
     __host__ __device__ static constexpr uint32_t part_bytes(int part) {            // per page
-        return kFp8 ? (part == kRope ? 1024u : (part == 0 ? 2048u + 64u : 2048u)) : 2048u;
+        return kFp8 ? (part == kRope ? 1024u : 8192u + 64u) : 2048u;
     }
     // exponent offset C and lazy threshold TAU of the softmax stabiliser, and
     // the headroom DELTA it is placed above a new maximum when it moves (so
@@ -115,21 +138,20 @@ struct Misc {
     uint64_t part_full[2][9], part_empty[2][9];   // per KV stage and part
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], pv_done[2];  // per P buffer: weights written / value MMAs of that buffer done
+    uint64_t q_full;          // the raw query rows of a piece landed
     uint64_t q_ready, o_free, drain;
+    uint64_t p_redo;          // a flagged tile's weights rewritten (all softmax warps)
+    uint32_t redo[2];         // per P buffer: gg + 1 when tile gg's weights must be rewritten
     uint64_t all_sync;        // all softmax warps (bounded waits, unlike bar.sync)
     uint64_t half_sync[kRowGroups];  // the four softmax warps of each row group
     uint32_t tmem_base;
     int abort;
     uint32_t stage_info[4];   // per tile mod 4: bit i page slot i loaded; bit 31 a page was invalid
-    int vote[kRowGroups][2][4];  // [row group][tile parity][warp]
     int col_lim[kN];          // positions visible to row r within this piece, 0 = none
     int col_bad[kN];
     float qscale;
     float amax[kSoftmaxWarps];
     float red[kRowGroups][4][kRpt];  // [row group][warp][row]
-    float m2c[kN];
-    float inv_l[kN];
-    float lse[kN];
 };
 
 template <bool kFp8>
@@ -143,10 +165,14 @@ __device__ __forceinline__ void cta_abort(const Problem &p, Misc &ms) {
 
 __device__ __forceinline__ bool aborted(Misc &ms) { return *reinterpret_cast<volatile int *>(&ms.abort) != 0; }
 
+// Bounded wait of a whole warp (all 32 lanes call it): every lane waits, and
+// the warp goes on only if every lane saw the phase, so a lane whose limit
+// runs out just before the phase completes cannot split the warp (the
+// .sync.aligned tensor-memory loads that follow need all of it).
 __device__ __forceinline__ bool waitb(const Problem &p, Misc &ms, uint64_t *bar, uint32_t parity) {
-    if (ptx::mbar_wait(bar, parity, kWaitLimit)) return true;
-    cta_abort(p, ms);
-    return false;
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, wait_limit(p)));
+    if (!ok) cta_abort(p, ms);
+    return ok;
 }
 
 // Barrier of a group of softmax warps: an mbarrier counting one arrival per
@@ -189,7 +215,8 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                          unsigned char *smem, Misc &ms, int slot) {
     using C = Cfg<kFp8>;
     const int lane = threadIdx.x & 31;
-    uint32_t g = 0;
+    uint32_t g = 0;            // tiles whose copies are all armed
+    uint32_t cur_parts = 0;    // parts of tile g armed so far (a stop can come mid-tile)
     bool first_piece = true;
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
@@ -226,28 +253,39 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                 const uint32_t pb = C::part_bytes(part) - (kFp8 && part == 0 && p.kv_scale_per_tensor ? 64u : 0u);
                 if (lane == 0) ptx::mbar_arrive_expect_tx(&ms.part_full[stage][part], n_ok * pb);
                 __syncwarp();
+                cur_parts = q + 1;
                 if (!ok) continue;
                 uint64_t *bar = &ms.part_full[stage][part];
                 if constexpr (kFp8) {
                     if (part == C::kRope) {
-                        ptx::tma_load_2d(st + 4 * C::kChunkBytes + lane * 1024, map_b, bar, 512, y);
+                        ptx::tma_load_2d(st + C::kRopeOff + lane * 1024, map_b, bar, 512, y);
                     } else {
-                        ptx::tma_load_2d(st + part * C::kChunkBytes + lane * 2048, map_a, bar, 128 * part, y);
-                        if (part == 0 && !p.kv_scale_per_tensor)
+                        // page slot `lane` = 8-position groups 2*lane, 2*lane+1
+                        ptx::tma_load_5d(st + lane * 2 * C::kGroupStride, map_a, bar, 0, 0, 0, 0, pid);
+                        if (!p.kv_scale_per_tensor)
                             ptx::bulk_load(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
                                            p.kv_scale + (int64_t)pid * kPage, 64, bar);
                     }
                 } else {
-                    ptx::tma_load_2d(st + part * C::kChunkBytes + lane * 2048, map_a, bar, 64 * part, y);
+                    ptx::tma_load_2d(st + part * C::kChunkStride + lane * 2048, map_a, bar, 64 * part, y);
                 }
             }
+            cur_parts = 0;
         }
         first_piece = false;
     });
-    // make sure no copy is still landing when the CTA leaves
-    for (uint32_t h = g > (uint32_t)C::kStages ? g - C::kStages : 0; h < g; ++h)
-        for (int part = 0; part < C::kParts; ++part)
-            ptx::mbar_wait(&ms.part_full[h % C::kStages][part], (h / C::kStages) & 1, kWaitLimit);
+    // Make sure no copy is still landing when the CTA leaves, also after a
+    // stop: a stage part is armed again only once its previous copy has been
+    // consumed, so only the last arming of each stage part can be in flight.
+    // Tiles 0..g-1 armed every part, tile g its first cur_parts parts.
+    for (int s2 = 0; s2 < C::kStages; ++s2) {
+        for (int qi = 0; qi < C::kParts; ++qi) {
+            const int part = qi == 0 ? C::kRope : qi - 1;
+            uint32_t n = g / C::kStages + ((uint32_t)s2 < g % C::kStages ? 1u : 0u);
+            if (g % C::kStages == (uint32_t)s2 && (uint32_t)qi < cur_parts) ++n;
+            if (n) ptx::mbar_wait(&ms.part_full[s2][part], (n - 1) & 1, kWaitLimit);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -266,15 +304,17 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
     constexpr uint32_t idesc_pv = kFp8 ? ptx::instr_desc(0, 0, 1, 1, kTileM, C::kNMma)
                                        : ptx::instr_desc(1, 1, 1, 1, kTileM, C::kNMma);
     uint32_t g = 0, pi = 0;
+    uint32_t redo_n = 0;       // rewrites of flagged tiles' weights consumed (lane 0)
 
     // Shared-memory descriptors are built once; an MMA then only adds the
     // byte offset of its operands (>> 4) to the start-address field.
     constexpr uint64_t kStageStep = (uint64_t)(C::kStageBytes >> 4);
-    const uint64_t dq_kv = ptx::smem_desc(kv0, 16, 1024, ptx::kSwizzle128B);       // K-major 128B chunks
+    const uint64_t dq_kv = ptx::smem_desc(kv0, 16, C::kGroupStride, ptx::kSwizzle128B);  // K-major 128B chunks
     const uint64_t dq_q = ptx::smem_desc(q0, 16, 1024, ptx::kSwizzle128B);
-    const uint64_t dr_kv = ptx::smem_desc(kv0 + 4 * C::kChunkBytes, 16, 512, ptx::kSwizzle64B);  // FP8 RoPE
+    const uint64_t dr_kv = ptx::smem_desc(kv0 + C::kRopeOff, 16, 512, ptx::kSwizzle64B);  // FP8 RoPE
     const uint64_t dr_q = ptx::smem_desc(q0 + C::kQRopeOff, 16, 512, ptx::kSwizzle64B);
-    const uint64_t dv_kv = ptx::smem_desc(kv0, 16384, 1024, ptx::kSwizzle128B);   // V^T, MN-major
+    // V^T, MN-major: 128-B atoms along the dims C::kChunkStride apart, 8-position groups along K
+    const uint64_t dv_kv = ptx::smem_desc(kv0, C::kChunkStride, C::kGroupStride, ptx::kSwizzle128B);
     const uint64_t dv_p = ptx::smem_desc(p0, 128, 2048, ptx::kSwizzleNone);       // P^T, MN-major
 
     // Score MMAs reading one part of the tile (accumulate from the second MMA of the tile on).
@@ -288,14 +328,17 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                 for (int ks = 0; ks < 2; ++ks)
                     ptx::mma_f8(d, dr_kv + so + 2 * ks, dr_q + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
             } else {
-                const uint64_t a = dq_kv + so + part * (C::kChunkBytes >> 4);
-                const uint64_t b = dq_q + part * (C::kQChunk >> 4);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_f8(d, a + 2 * ks, b + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
+                for (int c = 0; c < C::kDimChunks; ++c) {
+                    const uint64_t a = dq_kv + so + c * (C::kChunkStride >> 4);
+                    const uint64_t b = dq_q + c * (C::kQChunk >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        ptx::mma_f8(d, a + 2 * ks, b + 2 * ks, idesc_qk, (first && c == 0 && ks == 0) ? 0u : 1u);
+                }
             }
         } else {
-            const uint64_t a = dq_kv + so + part * (C::kChunkBytes >> 4);
+            const uint64_t a = dq_kv + so + part * (C::kChunkStride >> 4);
             const uint64_t b = dq_q + part * (C::kQChunk >> 4);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
@@ -313,29 +356,26 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
             const uint32_t d = tmem + C::kColO + C::kOStride * m;
             if constexpr (kFp8) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // 32 positions per MMA; N = 96: P hi | P lo
-                    ptx::mma_f8(d, a0 + m * (C::kChunkBytes >> 4) + ks * (4096 >> 4), pb + ks * (512 >> 4),
-                                idesc_pv, (first && ks == 0) ? 0u : 1u);
+                for (int ks = 0; ks < 4; ++ks)  // 32 positions (4 groups) per MMA; N = 96: P hi | P lo
+                    ptx::mma_f8(d, a0 + m * (C::kChunkStride >> 4) + ks * ((4 * C::kGroupStride) >> 4),
+                                pb + ks * (512 >> 4), idesc_pv, (first && ks == 0) ? 0u : 1u);
             } else {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)  // 16 positions per MMA
-                    ptx::mma_f16(d, a0 + 2 * m * (C::kChunkBytes >> 4) + ks * (2048 >> 4), pb + ks * (256 >> 4),
-                                 idesc_pv, (first && ks == 0) ? 0u : 1u);
-            }
-            if constexpr (kFp8) {
-                ptx::mma_commit(&ms.part_empty[stage][m]);
-            } else {
+                for (int ks = 0; ks < 8; ++ks)  // 16 positions (2 groups) per MMA
+                    ptx::mma_f16(d, a0 + 2 * m * (C::kChunkStride >> 4) + ks * ((2 * C::kGroupStride) >> 4),
+                                 pb + ks * (256 >> 4), idesc_pv, (first && ks == 0) ? 0u : 1u);
                 ptx::mma_commit(&ms.part_empty[stage][2 * m]);
                 ptx::mma_commit(&ms.part_empty[stage][2 * m + 1]);
             }
         }
+        if constexpr (kFp8) ptx::mma_commit(&ms.part_empty[stage][0]);
     };
 
     // Waits are made by lane 0 and broadcast, so the warp never diverges on
     // a phase that completes (or a limit that expires) while it waits.
     auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {
         int ok = 1;
-        if (lane == 0) ok = ptx::mbar_wait(bar, parity, kWaitLimit) && !aborted(ms);
+        if (lane == 0) ok = ptx::mbar_wait(bar, parity, wait_limit(p)) && !aborted(ms);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) cta_abort(p, ms);
         return ok != 0;
@@ -353,7 +393,8 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
         if (!wait1(&ms.q_ready, pi & 1)) return;
         int nq = 0, nv = 0;        // score / value groups issued
         int qp = 0;                // parts of tile nq seen landed
-        bool s_ok = false, o_ok = false;
+        bool s_ok = false, o_ok = false, p_ok = false;
+        int redo_state = 0;        // tile nv: 0 not read, 1 weights final, 2 being rewritten
         uint64_t t_idle = ptx::cycles();
         uint32_t spins = 0;
         while (nv < nt) {
@@ -363,7 +404,13 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                 if (nv < nq) {
                     const uint32_t gp = g0 + nv;
                     if (nv == 0 && !o_ok) o_ok = ptx::mbar_test(&ms.o_free, (pi & 1) ^ 1);
-                    if ((nv > 0 || o_ok) && ptx::mbar_test(&ms.p_full[gp & 1], (gp >> 1) & 1)) pick = 1;
+                    if ((nv > 0 || o_ok) && !p_ok) p_ok = ptx::mbar_test(&ms.p_full[gp & 1], (gp >> 1) & 1);
+                    if (p_ok) {
+                        // the flag was written before the last arrival on p_full
+                        if (redo_state == 0)
+                            redo_state = *reinterpret_cast<volatile uint32_t *>(&ms.redo[gp & 1]) == gp + 1 ? 2 : 1;
+                        if (redo_state == 1 || ptx::mbar_test(&ms.p_redo, redo_n & 1)) pick = 1;
+                    }
                 }
                 if (pick == 0 && nq < nt && nq <= nv + 1) {
                     const uint32_t gq = g0 + nq;
@@ -382,6 +429,9 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                 if (lane == 0) {
                     issue_pv(gp, nv == 0);
                     ptx::mma_commit(&ms.pv_done[gp & 1]);
+                    if (redo_state == 2) ++redo_n;
+                    p_ok = false;
+                    redo_state = 0;
                 }
                 __syncwarp();
                 ++nv;
@@ -408,7 +458,7 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
             }
             if (pick == 0 && (spins & 255) == 0) {
                 int expired = 0;
-                if (lane == 0) expired = (ptx::cycles() - t_idle > kWaitLimit) || aborted(ms);
+                if (lane == 0) expired = (ptx::cycles() - t_idle > wait_limit(p)) || aborted(ms);
                 if (__shfl_sync(0xffffffffu, expired, 0)) {
                     cta_abort(p, ms);
                     return;
@@ -427,39 +477,51 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
 // ---------------------------------------------------------------------------
 // warps 2-13: query staging, online softmax, epilogue
 // ---------------------------------------------------------------------------
-// Stages the 48 query rows of this group as the score MMA's B operand
-// (K-major, 128B / 64B swizzled chunks).  FP8: one pass into registers, the
-// block's largest |q| sets a power-of-two scale s, then hi = e4m3(q/s) goes to
-// rows 0-47 and lo = e4m3(q/s - hi) to rows 48-95.  A power-of-two s keeps q/s
-// a bf16 value, which hi + lo represents exactly (short of e4m3 underflow far
-// below the largest q).  Rows past R are zero.
+// The 48 query rows of a group arrive raw, as two bulk copies into the query
+// area: [48 rows][512] bf16 latent parts, then [48 rows][64] bf16 RoPE parts
+// (a sequence's rows are contiguous in q_lat and q_pe).  One thread issues
+// them when a piece starts, so they are in flight while the CTA sets up.
+constexpr int kQRawRope = kN * kDl * 2;   // byte offset of the raw RoPE rows
+
+__device__ __forceinline__ void issue_query_copy(const Problem &p, unsigned char *qs, Misc &ms, int b, int r0) {
+    const int rows = min(kN, p.R - r0);
+    const int64_t row0 = (int64_t)b * p.R + r0;
+    ptx::fence_proxy_async_smem();  // earlier generic writes to the area come first
+    ptx::mbar_arrive_expect_tx(&ms.q_full, (uint32_t)rows * (kDl + kDr) * 2);
+    ptx::bulk_load(qs, p.q_lat + row0 * kDl, (uint32_t)rows * kDl * 2, &ms.q_full);
+    ptx::bulk_load(qs + kQRawRope, p.q_pe + row0 * kDr, (uint32_t)rows * kDr * 2, &ms.q_full);
+}
+
+// Turns the raw rows into the score MMA's B operand in place (K-major, 128B /
+// 64B swizzled chunks): every thread reads its units into registers, a
+// barrier of all softmax warps separates the reads from the writes, then the
+// units are written back in operand layout.  FP8: the block's largest |q|
+// sets a power-of-two scale s, hi = e4m3(q/s) goes to rows 0-47 and lo =
+// e4m3(q/s - hi) to rows 48-95.  A power-of-two s keeps q/s a bf16 value,
+// which hi + lo represents exactly (short of e4m3 underflow far below the
+// largest q).  Rows past R are zero.
 template <bool kFp8>
-__device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int b, int r0, int st,
-                           GroupSync &gsync) {
+__device__ bool stage_query(const Problem &p, unsigned char *smem, Misc &ms, int r0, int st, GroupSync &gsync) {
     using C = Cfg<kFp8>;
-    const int64_t qrow0 = (int64_t)b * p.R;
     unsigned char *qs = smem + C::kQOff;
+    const int rows = min(kN, p.R - r0);
     if constexpr (kFp8) {
         // unit = 16 consecutive dims of one row (36 units per row, 32 latent + 4 RoPE)
         constexpr int kUnits = kN * 36;
         constexpr int kPer = (kUnits + kSoftmaxThreads - 1) / kSoftmaxThreads;  // 7
         uint4 v[kPer][2];
         float amax = 0.f;
-        // every load is issued before any is used: one memory round trip
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int u = st + j * kSoftmaxThreads;
             const int row = u / 36, uu = u % 36;
             v[j][0] = v[j][1] = make_uint4(0, 0, 0, 0);
-            if (u < kUnits && r0 + row < p.R) {
-                const __nv_bfloat16 *src = uu < 32 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 16
-                                                   : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 32) * 16;
-                v[j][0] = __ldg(reinterpret_cast<const uint4 *>(src));
-                v[j][1] = __ldg(reinterpret_cast<const uint4 *>(src) + 1);
+            if (u < kUnits && row < rows) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    uu < 32 ? qs + row * (kDl * 2) + uu * 32 : qs + kQRawRope + row * (kDr * 2) + (uu - 32) * 32);
+                v[j][0] = src[0];
+                v[j][1] = src[1];
             }
-        }
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v[j][h]);
@@ -472,7 +534,7 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
         }
         amax = warp_max(amax);
         if ((threadIdx.x & 31) == 0) ms.amax[(threadIdx.x >> 5) - 2] = amax;
-        if (!gsync(p, ms)) return false;
+        if (!gsync(p, ms)) return false;   // also: every raw read is done
 #pragma unroll
         for (int w = 0; w < kSoftmaxWarps; ++w) amax = fmaxf(amax, ms.amax[w]);
         int e2 = 0;
@@ -491,13 +553,13 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {  // 4 dims -> one 32-bit word of hi and of lo
                     const float2 f0 = __bfloat1622float2(b2[2 * q]), f1 = __bfloat1622float2(b2[2 * q + 1]);
-                    const float x0 = f0.x * inv, x1 = f0.y * inv, x2 = f1.x * inv, x3 = f1.y * inv;
-                    const uint32_t h01 = ptx::e4m3x2(x0, x1), h23 = ptx::e4m3x2(x2, x3);
-                    float a0, a1, a2, a3;
-                    ptx::e4m3x2_to_f32(h01, &a0, &a1);
-                    ptx::e4m3x2_to_f32(h23, &a2, &a3);
+                    // q/s is exact in f16 down to its subnormals, far below lo's e4m3 range
+                    const uint32_t p01 = ptx::f16x2(f0.x * inv, f0.y * inv), p23 = ptx::f16x2(f1.x * inv, f1.y * inv);
+                    const uint32_t h01 = ptx::e4m3x2_from_f16x2(p01), h23 = ptx::e4m3x2_from_f16x2(p23);
+                    const uint32_t l01 = ptx::e4m3x2_from_f16x2(ptx::sub_f16x2(p01, ptx::f16x2_from_e4m3x2(h01)));
+                    const uint32_t l23 = ptx::e4m3x2_from_f16x2(ptx::sub_f16x2(p23, ptx::f16x2_from_e4m3x2(h23)));
                     hw[2 * h + q] = h01 | (h23 << 16);
-                    lw[2 * h + q] = ptx::e4m3x2(x0 - a0, x1 - a1) | (ptx::e4m3x2(x2 - a2, x3 - a3) << 16);
+                    lw[2 * h + q] = l01 | (l23 << 16);
                 }
             }
             const uint4 hi4 = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -515,29 +577,25 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
         }
     } else {
         constexpr int kUnits = kN * 72;  // 8 dims per unit
-        constexpr int kPer = (kUnits + 2 * kSoftmaxThreads - 1) / (2 * kSoftmaxThreads);  // 7 per batch
-#pragma unroll 1
-        for (int batch = 0; batch < 2; ++batch) {
-            uint4 v[kPer];
+        constexpr int kPer = (kUnits + kSoftmaxThreads - 1) / kSoftmaxThreads;  // 9
+        uint4 v[kPer];
 #pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int u = st + (batch * kPer + j) * kSoftmaxThreads;
-                const int row = u / 72, uu = u % 72;
-                v[j] = make_uint4(0, 0, 0, 0);
-                if (u < kUnits && r0 + row < p.R) {
-                    const __nv_bfloat16 *src = uu < 64 ? p.q_lat + (qrow0 + r0 + row) * kDl + uu * 8
-                                                       : p.q_pe + (qrow0 + r0 + row) * kDr + (uu - 64) * 8;
-                    v[j] = __ldg(reinterpret_cast<const uint4 *>(src));
-                }
-            }
+        for (int j = 0; j < kPer; ++j) {
+            const int u = st + j * kSoftmaxThreads;
+            const int row = u / 72, uu = u % 72;
+            v[j] = make_uint4(0, 0, 0, 0);
+            if (u < kUnits && row < rows)
+                v[j] = *reinterpret_cast<const uint4 *>(uu < 64 ? qs + row * (kDl * 2) + uu * 16
+                                                                : qs + kQRawRope + row * (kDr * 2) + (uu - 64) * 16);
+        }
+        if (!gsync(p, ms)) return false;   // every raw read is done
 #pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int u = st + (batch * kPer + j) * kSoftmaxThreads;
-                if (u >= kUnits) continue;
-                const int row = u / 72, uu = u % 72;
-                const int c = uu >> 3, k = uu & 7;
-                *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4)) = v[j];
-            }
+        for (int j = 0; j < kPer; ++j) {
+            const int u = st + j * kSoftmaxThreads;
+            if (u >= kUnits) continue;
+            const int row = u / 72, uu = u % 72;
+            const int c = uu >> 3, k = uu & 7;
+            *reinterpret_cast<uint4 *>(qs + c * C::kQChunk + row * 128 + ((k ^ (row & 7)) << 4)) = v[j];
         }
     }
     return true;
@@ -547,12 +605,14 @@ __device__ bool load_query(const Problem &p, unsigned char *smem, Misc &ms, int 
 // (48 columns apart) are added.
 template <bool kFp8>
 __device__ __forceinline__ void tmem_rows(uint32_t taddr, float *v) {
-    ptx::tmem_ld_cols<kRpt>(taddr, v);
     if constexpr (kFp8) {
+        static_assert(kRpt == 16, "the paired load takes 16 columns per half");
         float w[kRpt];
-        ptx::tmem_ld_cols<kRpt>(taddr + kN, w);
+        ptx::tmem_ld16_pair(taddr, taddr + kN, v, w);
 #pragma unroll
         for (int c = 0; c < kRpt; ++c) v[c] += w[c];
+    } else {
+        ptx::tmem_ld_cols<kRpt>(taddr, v);
     }
 }
 
@@ -576,9 +636,16 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
     GroupSync all_sync(&ms.all_sync), hsync(&ms.half_sync[h]);
     const float static_scale = kFp8 && p.kv_scale_per_tensor ? __ldg(p.kv_scale) : 1.f;
 
+    uint32_t qn = 0;           // query copies waited for (phase of q_full)
+    uint32_t q_issued = 0;     // query copies issued (thread st == 0)
     for_each_piece(p, slot, [&](const Piece &pc) {
         if (aborted(ms)) return;
         const int nt = ntiles_of(pc);
+        // the query rows go out first, so they land while the piece is set up
+        if (nt > 0 && st == 0) {
+            issue_query_copy(p, smem + C::kQOff, ms, pc.b, r0);
+            ++q_issued;
+        }
         // visible positions per row, limited to this piece's pages
         if (st < kN) {
             const int r = r0 + st;
@@ -614,7 +681,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             return;
         }
 
-        if (!load_query<kFp8>(p, smem, ms, pc.b, r0, st, all_sync)) return;
+        if (!waitb(p, ms, &ms.q_full, qn & 1)) return;
+        ++qn;
+        if (!stage_query<kFp8>(p, smem, ms, r0, st, all_sync)) return;
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ms.q_ready);
@@ -630,6 +699,61 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         }
         bool piece_bad = false;
         const uint32_t g0 = g;
+
+        // This thread's entries of the tile's weight operand P: e = ex2(s - m2c)
+        // for its kRpt rows (times the token's value scale for FP8), written to
+        // P buffer gg & 1 in the layout the value MMA reads.  With add_sums the
+        // weights also enter the row sums.
+        auto store_p = [&](const float (&sc)[kRpt], float kvs, bool add_sums, uint32_t gg) {
+            unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
+            if constexpr (kFp8) {
+                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of this
+                // thread's rows.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
+                // far below lo's 2^-9), hi = e4m3(p16), and p16 - hi is exact in
+                // f16, so lo = e4m3(p16 - hi).
+#pragma unroll
+                for (int w = 0; w < kRpt / 4; ++w) {
+                    uint32_t hp[2], lp[2];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int c0 = 4 * w + 2 * q;
+                        const float e0 = ptx::ex2(sc[c0] - m2c[c0]), e1 = ptx::ex2(sc[c0 + 1] - m2c[c0 + 1]);
+                        if (add_sums) {
+                            lsum[c0] += e0;
+                            lsum[c0 + 1] += e1;
+                        }
+                        const uint32_t p16 = ptx::f16x2(e0 * kvs, e1 * kvs);
+                        hp[q] = ptx::e4m3x2_from_f16x2(p16);
+                        lp[q] = ptx::e4m3x2_from_f16x2(ptx::sub_f16x2(p16, ptx::f16x2_from_e4m3x2(hp[q])));
+                    }
+                    // P^T is [16-row groups of 16 B] x 128 positions; each four of this
+                    // thread's rows lie in one group
+                    const int row0 = cb + 4 * w;
+                    const int off = (row0 >> 4) * 2048 + i * 16 + (row0 & 15);
+                    *reinterpret_cast<uint32_t *>(pb + off) = hp[0] | (hp[1] << 16);
+                    *reinterpret_cast<uint32_t *>(pb + C::kPLoOff + off) = lp[0] | (lp[1] << 16);
+                }
+            } else {
+                // bf16 P^T: [8-row groups of 16 B] x 128 positions, two rows per word
+#pragma unroll
+                for (int w = 0; w < kRpt / 2; ++w) {
+                    const int c0 = 2 * w;
+                    const float e0 = ptx::ex2(sc[c0] - m2c[c0]), e1 = ptx::ex2(sc[c0 + 1] - m2c[c0 + 1]);
+                    if (add_sums) {
+                        lsum[c0] += e0;
+                        lsum[c0 + 1] += e1;
+                    }
+                    const int row0 = cb + c0;
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+                    *reinterpret_cast<uint32_t *>(pb + (row0 >> 3) * 2048 + i * 16 + 2 * (row0 & 7)) =
+                        *reinterpret_cast<uint32_t *>(&b2);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncwarp();
+        };
+
         for (int k = 0; k < nt; ++k) {
             const uint32_t gg = g0 + k;
             const int stage = gg % C::kStages;
@@ -637,17 +761,6 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             if (!waitb(p, ms, &ms.part_full[stage][0], (gg / C::kStages) & 1)) return;
             const uint32_t info = ms.stage_info[gg & 3];
             piece_bad |= (info >> 31) != 0;
-            const int sb = gg % C::kSBufs;
-            if (!waitb(p, ms, &ms.s_full[sb], (gg / C::kSBufs) & 1)) return;
-            ptx::tc_fence_after();
-            float s[kRpt];
-            tmem_rows<kFp8>(tmem + (sb ? C::kColS1 : 0u) + cb, s);
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&ms.s_free[sb]);
-            // P buffer gg & 1 is free once the value MMAs of tile gg - 2 are done
-            if (gg >= 2 && !waitb(p, ms, &ms.pv_done[gg & 1], ((gg - 2) >> 1) & 1)) return;
-
             const int pos0 = (pc.page_lo + k * kTilePages) * kPage;
             const int pos = pos0 + i;
             const bool loaded = (info >> (i / kPage)) & 1u;
@@ -663,6 +776,16 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             const bool fast = (info & 0xFFu) == 0xFFu && pos0 + kTileM <= min_lim;
             // u = s + lkvs exceeds the stabiliser by more than TAU iff s > m2c + (C + TAU - lkvs)
             const float kx = C::kC + C::kTau - lkvs;
+
+            const int sb = gg % C::kSBufs;
+            if (!waitb(p, ms, &ms.s_full[sb], (gg / C::kSBufs) & 1)) return;
+            ptx::tc_fence_after();
+            float s[kRpt];
+            tmem_rows<kFp8>(tmem + (sb ? C::kColS1 : 0u) + cb, s);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ms.s_free[sb]);
+
             bool exceed = false;
 #pragma unroll
             for (int c = 0; c < kRpt; ++c) {
@@ -670,111 +793,77 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 s[c] = valid ? s[c] * factor : -INFINITY;       // score, log2 units
                 exceed |= s[c] > m2c[c] + kx;
             }
-            // all lanes of the row group must agree on the stabiliser
-            const int vote = __any_sync(0xffffffffu, exceed);
-            if (lane == 0) ms.vote[h][gg & 1][w4] = vote;
-            if (!hsync(p, ms)) return;
-            const int *vv = ms.vote[h][gg & 1];
-            if (vv[0] | vv[1] | vv[2] | vv[3]) {
-#pragma unroll
-                for (int c = 0; c < kRpt; ++c) {
-                    const float cm = warp_max(s[c] + lkvs);
-                    if (lane == 0) ms.red[h][w4][c] = cm;
-                }
-                if (!hsync(p, ms)) return;
-                float alpha[kRpt];
-                bool moved = false;
-#pragma unroll
-                for (int c = 0; c < kRpt; ++c) {
-                    const float cm = fmaxf(fmaxf(ms.red[h][0][c], ms.red[h][1][c]),
-                                           fmaxf(ms.red[h][2][c], ms.red[h][3][c]));
-                    const float old = m2c[c] + C::kC;
-                    const float mn = cm > old + C::kTau ? cm + C::kDelta : old;
-                    alpha[c] = mn == old ? 1.f : ptx::ex2(old - mn);
-                    moved |= mn != old;
-                    m2c[c] = mn - C::kC;
-                    lsum[c] *= alpha[c];
-                }
-                if (!hsync(p, ms)) return;  // red[] reads done before any reuse
-                if (moved && k > 0) {
-                    // O^T holds earlier tiles: wait for their value MMA, then rescale rows
-                    if (!waitb(p, ms, &ms.pv_done[(gg - 1) & 1], ((gg - 1) >> 1) & 1)) return;
-                    ptx::tc_fence_after();
-#pragma unroll 1
-                    for (int m = 0; m < 4; ++m) {
-#pragma unroll 1
-                        for (int part = 0; part < (kFp8 ? 2 : 1); ++part) {
-                            float o[kRpt];
-                            const uint32_t oc = tmem + C::kColO + C::kOStride * m + part * kN + cb;
-                            ptx::tmem_ld_cols<kRpt>(oc, o);
-#pragma unroll
-                            for (int c = 0; c < kRpt; ++c) o[c] *= alpha[c];
-                            ptx::tmem_st_cols<kRpt>(oc, o);
-                        }
-                    }
-                }
-            }
-            // weights e = ex2(s - m2c) enter the row sums; the value MMA takes
-            // e times the token's value scale (FP8) as its P entry
-#pragma unroll
-            for (int c = 0; c < kRpt; ++c) {
-                const float e = ptx::ex2(s[c] - m2c[c]);
-                lsum[c] += e;
-                s[c] = kFp8 ? e * kvs : e;
-            }
-            // rows past the context in a loaded page may hold anything; their
-            // weight is 0 but 0 * NaN is NaN, so clear them before the value MMA
-            if (h == 0 && !fast && loaded && pos >= pc.ctx) {
+            // Optimistic stabiliser: every warp writes its weights with the
+            // current stabiliser and flags the tile if one of them would be too
+            // large; the tile's fate is read once every warp has written it.
+            const bool wex = __any_sync(0xffffffffu, exceed);
+            // P buffer gg & 1 is free once the value MMAs of tile gg - 2 are done;
+            // the MMA warp read that tile's flag (same slot) before issuing them
+            if (gg >= 2 && !waitb(p, ms, &ms.pv_done[gg & 1], ((gg - 2) >> 1) & 1)) return;
+            if (wex && lane == 0) *reinterpret_cast<volatile uint32_t *>(&ms.redo[gg & 1]) = gg + 1;
+            // rows past the context, and page slots this tile did not load, may
+            // hold anything; their weight is 0 but 0 * NaN is NaN, so clear
+            // their values before the value MMA
+            if (h == 0 && !fast && (!loaded || pos >= pc.ctx)) {
                 unsigned char *stg = smem + C::kKvOff + stage * C::kStageBytes;
 #pragma unroll
-                for (int c = 0; c < C::kVChunks; ++c) {
-                    uint4 *row = reinterpret_cast<uint4 *>(stg + c * C::kChunkBytes + i * 128);
+                for (int c = 0; c < C::kDimChunks; ++c) {
+                    uint4 *row = reinterpret_cast<uint4 *>(stg + (i >> 3) * C::kGroupStride + c * C::kChunkStride +
+                                                           (i & 7) * 128);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) row[e] = make_uint4(0, 0, 0, 0);
                 }
             }
-            unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
-            if constexpr (kFp8) {
-                // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of this
-                // thread's rows.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
-                // far below lo's 2^-9), hi = e4m3(p16), and p16 - hi is exact in
-                // f16, so lo = e4m3(p16 - hi).
-                uint32_t hw[kRpt / 4], lw[kRpt / 4];
+            // a flagged warp's weights are rewritten below, and its sums added then
+            store_p(s, kvs, !wex, gg);
+            if (lane == 0) ptx::mbar_arrive(&ms.p_full[gg & 1]);
+
+            // every warp has written its weights and its flag for tile gg
+            if (!waitb(p, ms, &ms.p_full[gg & 1], (gg >> 1) & 1)) return;
+            if (*reinterpret_cast<volatile uint32_t *>(&ms.redo[gg & 1]) != gg + 1) continue;
+
+            // Slow path (the first tile of a piece, then rarely): move the
+            // stabiliser of the rows whose weights overflowed to DELTA above
+            // their new maximum, rescale what came before, rewrite P.  The
+            // value MMAs of this tile wait for it (p_redo).
 #pragma unroll
-                for (int w = 0; w < kRpt / 4; ++w) {
-                    uint32_t hp[2], lp[2];
+            for (int c = 0; c < kRpt; ++c) {
+                const float cm = warp_max(s[c] + lkvs);
+                if (lane == 0) ms.red[h][w4][c] = cm;
+            }
+            if (!all_sync(p, ms)) return;
+            float alpha[kRpt];
+            bool moved = false;
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint32_t p16 = ptx::f16x2(s[4 * w + 2 * q], s[4 * w + 2 * q + 1]);
-                        hp[q] = ptx::e4m3x2_from_f16x2(p16);
-                        lp[q] = ptx::e4m3x2_from_f16x2(ptx::sub_f16x2(p16, ptx::f16x2_from_e4m3x2(hp[q])));
+            for (int c = 0; c < kRpt; ++c) {
+                const float cm = fmaxf(fmaxf(ms.red[h][0][c], ms.red[h][1][c]),
+                                       fmaxf(ms.red[h][2][c], ms.red[h][3][c]));
+                const float old = m2c[c] + C::kC;
+                const float mn = cm > old + C::kTau ? cm + C::kDelta : old;
+                alpha[c] = mn == old ? 1.f : ptx::ex2(old - mn);
+                moved |= mn != old;
+                m2c[c] = mn - C::kC;
+                lsum[c] *= alpha[c];     // earlier tiles, and this one for unflagged warps
+            }
+            if (moved && k > 0) {
+                // O^T holds earlier tiles: wait for their value MMA, then rescale rows
+                if (!waitb(p, ms, &ms.pv_done[(gg - 1) & 1], ((gg - 1) >> 1) & 1)) return;
+                ptx::tc_fence_after();
+#pragma unroll 1
+                for (int m = 0; m < 4; ++m) {
+#pragma unroll 1
+                    for (int part = 0; part < (kFp8 ? 2 : 1); ++part) {
+                        float o[kRpt];
+                        const uint32_t oc = tmem + C::kColO + C::kOStride * m + part * kN + cb;
+                        ptx::tmem_ld_cols<kRpt>(oc, o);
+#pragma unroll
+                        for (int c = 0; c < kRpt; ++c) o[c] *= alpha[c];
+                        ptx::tmem_st_cols<kRpt>(oc, o);
                     }
-                    hw[w] = hp[0] | (hp[1] << 16);
-                    lw[w] = lp[0] | (lp[1] << 16);
-                }
-                // P^T is [16-row groups of 16 B] x 128 positions; each four of this
-                // thread's rows lie in one group
-#pragma unroll
-                for (int w = 0; w < kRpt / 4; ++w) {
-                    const int row0 = cb + 4 * w;
-                    const int off = (row0 >> 4) * 2048 + i * 16 + (row0 & 15);
-                    *reinterpret_cast<uint32_t *>(pb + off) = hw[w];
-                    *reinterpret_cast<uint32_t *>(pb + C::kPLoOff + off) = lw[w];
-                }
-            } else {
-                // bf16 P^T: [8-row groups of 16 B] x 128 positions, two rows per word
-#pragma unroll
-                for (int w = 0; w < kRpt / 2; ++w) {
-                    const int row0 = cb + 2 * w;
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(s[2 * w], s[2 * w + 1]);
-                    *reinterpret_cast<uint32_t *>(pb + (row0 >> 3) * 2048 + i * 16 + 2 * (row0 & 7)) =
-                        *reinterpret_cast<uint32_t *>(&b2);
                 }
             }
-            ptx::fence_proxy_async_smem();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&ms.p_full[gg & 1]);
+            store_p(s, kvs, wex, gg);
+            if (lane == 0) ptx::mbar_arrive(&ms.p_redo);
         }
         g = g0 + nt;
 
@@ -787,37 +876,33 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             const float v = warp_sum(lsum[c]);
             if (lane == 0) ms.red[h][w4][c] = v;
         }
-        if (hst == 0) {
-#pragma unroll
-            for (int c = 0; c < kRpt; ++c) ms.m2c[cb + c] = m2c[c];
-        }
         if (!hsync(p, ms)) return;
-        if (hst < kRpt) {
-            const int col = cb + hst;
-            const float l = ms.red[h][0][hst] + ms.red[h][1][hst] + ms.red[h][2][hst] + ms.red[h][3][hst];
-            const bool bad = piece_bad || ms.col_bad[col];
-            // ln sum_j exp(score_j) = (m2c + log2 l) * ln 2
-            ms.inv_l[col] = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
-            ms.lse[col] = bad ? NAN : (l > 0.f ? (ms.m2c[col] + __log2f(l)) * kLn2 : -INFINITY);
-        }
-        if (!hsync(p, ms)) return;
-        const int ncols = min(kRpt, rows_here - cb);
-        // O goes out one 128-dim block at a time: every thread writes its dim of
-        // its row group's rows into a [48 rows][128] staging box (the query area is
-        // free until the next piece), then one thread stores the box with a
-        // tensor store.  The maps clip rows past the sequence's R, and two
-        // staging boxes alternate so the next block is written while the
-        // previous one is copied out.
+        // every thread forms the sums of its own rows; thread hst < kRpt of the
+        // group also forms row cb + hst's log-sum-exp
         float inv_l[kRpt];
+        float row_lse = 0.f;
 #pragma unroll
-        for (int c = 0; c < kRpt; ++c) inv_l[c] = ms.inv_l[cb + c];
+        for (int c = 0; c < kRpt; ++c) {
+            const float l = ms.red[h][0][c] + ms.red[h][1][c] + ms.red[h][2][c] + ms.red[h][3][c];
+            const bool bad = piece_bad || ms.col_bad[cb + c];
+            inv_l[c] = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+            // ln sum_j exp(score_j) = (m2c + log2 l) * ln 2
+            if (c == hst) row_lse = bad ? NAN : (l > 0.f ? (m2c[c] + __log2f(l)) * kLn2 : -INFINITY);
+        }
+        // O goes out one 128-dim block at a time, each row group on its own:
+        // the group's threads write their dims of its 16 rows into a [16][128]
+        // staging box (two per group alternate, in the query area, free until
+        // the next piece), and the group's first thread stores the box with a
+        // tensor store; the maps clip rows past the sequence's R.
+        const int nrows = min(kRpt, rows_here - cb);
         const bool f32_box = !pc.single || p.out_f32;
-        constexpr int kBoxBytes = kN * 128 * 4;
+        constexpr int kBoxBytes = kRpt * 128 * 4;
+#pragma unroll 1
         for (int m = 0; m < 4; ++m) {
-            unsigned char *box = smem + C::kQOff + (m & 1) * kBoxBytes;
+            unsigned char *box = smem + C::kQOff + (2 * h + (m & 1)) * kBoxBytes;
             if (m >= 2) {  // the store of block m - 2 has finished reading this box
-                if (st == 0) ptx::bulk_wait_read<1>();
-                if (!all_sync(p, ms)) return;
+                if (hst == 0) ptx::bulk_wait_read<1>();
+                if (!hsync(p, ms)) return;
             }
             float o[kRpt];
             tmem_rows<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
@@ -825,27 +910,27 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             for (int c = 0; c < kRpt; ++c) {
                 const float v = o[c] * inv_l[c];
                 if (f32_box)
-                    reinterpret_cast<float *>(box)[(cb + c) * 128 + i] = v;
+                    reinterpret_cast<float *>(box)[c * 128 + i] = v;
                 else
-                    reinterpret_cast<__nv_bfloat16 *>(box)[(cb + c) * 128 + i] = __float2bfloat16_rn(v);
+                    reinterpret_cast<__nv_bfloat16 *>(box)[c * 128 + i] = __float2bfloat16_rn(v);
             }
             ptx::fence_proxy_async_smem();
-            if (!all_sync(p, ms)) return;
-            if (st == 0) {
+            if (!hsync(p, ms)) return;
+            if (hst == 0 && nrows > 0) {
                 if (pc.single)
-                    ptx::tma_store_3d(map_out, box, 128 * m, r0, pc.b);
+                    ptx::tma_store_3d(map_out, box, 128 * m, r0 + cb, pc.b);
                 else
-                    ptx::tma_store_3d(map_part, box, 128 * m, (int)pc.piece, r0);
+                    ptx::tma_store_3d(map_part, box, 128 * m, (int)pc.piece, r0 + cb);
                 ptx::bulk_commit();
             }
         }
-        if (st == 0) ptx::bulk_wait_read<0>();  // boxes read before the query area is reused
-        if (hst < ncols) {
+        if (hst == 0) ptx::bulk_wait_read<0>();  // boxes read before the query area is reused
+        if (hst < nrows) {
             const int64_t r = r0 + cb + hst;
             if (pc.single) {
-                if (p.lse) p.lse[(int64_t)pc.b * p.R + r] = ms.lse[cb + hst];
+                if (p.lse) p.lse[(int64_t)pc.b * p.R + r] = row_lse;
             } else {
-                p.part_lse[r * p.max_pieces + pc.piece] = ms.lse[cb + hst];
+                p.part_lse[r * p.max_pieces + pc.piece] = row_lse;
             }
         }
         ptx::tc_fence_before();
@@ -853,6 +938,10 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         if (lane == 0) ptx::mbar_arrive(&ms.o_free);
         all_sync(p, ms);  // smem per-piece state reused next piece
     });
+    // after a stop, a query copy may still be landing and an output store may
+    // still be reading its staging box
+    if (st == 0 && q_issued > qn) ptx::mbar_wait(&ms.q_full, (q_issued - 1) & 1, kWaitLimit);
+    if (hst == 0) ptx::bulk_wait_read<0>();
 }
 
 template <bool kFp8>
@@ -868,11 +957,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int slot = blockIdx.x / p.n_groups;
     const int g_idx = blockIdx.x % p.n_groups;
+    // the merge kernel that follows may be scheduled now; it waits for this
+    // grid to finish before it reads anything this grid writes
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    // Zero the KV stages once: rows never loaded then hold finite values.
-    for (int o = threadIdx.x * 16; o < C::kStages * C::kStageBytes; o += kThreads * 16)
-        *reinterpret_cast<uint4 *>(smem + C::kKvOff + o) = make_uint4(0, 0, 0, 0);
-    ptx::fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             for (int q = 0; q < 9; ++q) {
@@ -888,9 +976,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&ms.pv_done[b], 1);
         }
         ptx::mbar_init(&ms.q_ready, kSoftmaxWarps);
+        ptx::mbar_init(&ms.q_full, 1);
         ptx::mbar_init(&ms.o_free, kSoftmaxWarps);
         ptx::mbar_init(&ms.drain, 1);
         ptx::mbar_init(&ms.all_sync, kSoftmaxWarps);
+        ptx::mbar_init(&ms.p_redo, kSoftmaxWarps);
+        ms.redo[0] = ms.redo[1] = 0;
         ms.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -921,16 +1012,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// The driver's tensor-map encoder, looked up once (a function-local static is
+// initialised exactly once even when several host threads call at once).
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -950,8 +1043,25 @@ bool make_kv_map(CUtensorMap *map, const void *base, int num_pages, bool fp8, ui
     return r == CUDA_SUCCESS;
 }
 
-// Output views for the epilogue's tensor stores, boxes of 128 dims x 48 rows:
-// out as [B][R][512] (bf16 or fp32), the partials as [R][pieces][512] fp32.
+// 5-D view of the FP8 pool's c_kv bytes: {128 bytes of a chunk, 8 rows, 4
+// chunks, 2 halves of a page, pages}, one box = one page's 512 latent bytes,
+// landing as [half][chunk][8 rows][128 B] (the MMA's swizzled K-major atoms).
+bool make_fp8_latent_map(CUtensorMap *map, const void *base, int num_pages) {
+    auto encode = get_encode_fn();
+    if (!encode) return false;
+    const cuuint64_t dims[5] = {128, 8, 4, 2, (cuuint64_t)num_pages};
+    const cuuint64_t strides[4] = {(cuuint64_t)kD, 128, (cuuint64_t)8 * kD, (cuuint64_t)kPage * kD};
+    const cuuint32_t box[5] = {128, 8, 4, 2, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Output views for the epilogue's tensor stores, boxes of 128 dims x 16 rows
+// (one softmax row group): out as [B][R][512] (bf16 or fp32), the partials
+// as [R][pieces][512] fp32.
 bool make_out_maps(CUtensorMap *mo, CUtensorMap *mp, const Problem &p) {
     auto encode = get_encode_fn();
     if (!encode) return false;
@@ -960,7 +1070,7 @@ bool make_out_maps(CUtensorMap *mo, CUtensorMap *mp, const Problem &p) {
     {
         const cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)p.R, (cuuint64_t)p.B};
         const cuuint64_t strides[2] = {(cuuint64_t)kDl * osz, (cuuint64_t)p.R * kDl * osz};
-        const cuuint32_t box[3] = {128, (cuuint32_t)kN, 1};
+        const cuuint32_t box[3] = {128, (cuuint32_t)kRpt, 1};
         if (encode(mo, p.out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.out, dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -972,7 +1082,7 @@ bool make_out_maps(CUtensorMap *mo, CUtensorMap *mp, const Problem &p) {
     }
     const cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)p.max_pieces, (cuuint64_t)p.R};
     const cuuint64_t strides[2] = {(cuuint64_t)kDl * 4, (cuuint64_t)p.max_pieces * kDl * 4};
-    const cuuint32_t box[3] = {128, 1, (cuuint32_t)kN};
+    const cuuint32_t box[3] = {128, 1, (cuuint32_t)kRpt};
     return encode(mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.part_o, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -983,7 +1093,7 @@ int launch_impl(const Problem &p, cudaStream_t stream) {
     CUtensorMap ma, mb, mo, mp;
     bool ok;
     if (kFp8) {
-        ok = make_kv_map(&ma, p.kv, p.num_pages, true, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        ok = make_fp8_latent_map(&ma, p.kv, p.num_pages) &&
              make_kv_map(&mb, p.kv, p.num_pages, true, 64, CU_TENSOR_MAP_SWIZZLE_64B);
     } else {
         ok = make_kv_map(&ma, p.kv, p.num_pages, false, 64, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -1005,8 +1115,8 @@ int launch_impl(const Problem &p, cudaStream_t stream) {
 }
 
 static_assert(smem_bytes<true>() <= 232448, "FP8 tile does not fit shared memory");
-static_assert(2 * kN * 128 * 4 <= Cfg<true>::kQBytes && 2 * kN * 128 * 4 <= Cfg<false>::kQBytes,
-              "two epilogue staging boxes must fit the query area");
+static_assert(2 * kRowGroups * kRpt * 128 * 4 <= Cfg<true>::kQBytes && 2 * kRowGroups * kRpt * 128 * 4 <= Cfg<false>::kQBytes,
+              "each row group's two epilogue staging boxes must fit the query area");
 static_assert(smem_bytes<false>() <= 232448, "bf16 tile does not fit shared memory");
 static_assert(Cfg<true>::kColO + 3 * Cfg<true>::kOStride + Cfg<true>::kNMma <= kTmemCols, "TMEM overflow");
 static_assert(Cfg<false>::kColO + 3 * Cfg<false>::kOStride + Cfg<false>::kNMma <= kTmemCols, "TMEM overflow");

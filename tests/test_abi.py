@@ -61,6 +61,7 @@ BAD_DIMS = [dict(B=0), dict(T=0), dict(T=9), dict(H=0), dict(T=8, H=129), dict(n
             dict(out_dtype=5), dict(num_splits=-1), dict(kernel=7),
             dict(B=1 << 26, T=8, H=1),                 # 2^29 query rows: past the merge grid
             dict(kv_scale_per_tensor=2), dict(kv_scale_per_tensor=1),  # the latter with a bf16 cache
+            dict(wait_limit_kcycles=-1),
             # B * max_pages_per_seq = 2^32 page slots: past the device schedule's 32-bit sums
             dict(B=1 << 20, max_pages_per_seq=1 << 12, page_table_stride=1 << 12)]
 
@@ -142,6 +143,7 @@ int main(void) {
     printf("sizeof %zu\n", sizeof(mla_dims));
     F(B) F(T) F(H) F(num_pages) F(max_pages_per_seq) F(page_table_stride) F(kv_dtype)
     F(out_dtype) F(num_splits) F(kernel) F(vis_lens) F(stage_event) F(kv_scale_per_tensor)
+    F(wait_limit_kcycles)
     return 0;
 }
 """
