@@ -87,7 +87,7 @@ int make_plan(const mla_dims *d, Plan *pl) {
     pl->max_pieces = pl->n_slots > 1 ? (int64_t)pl->n_slots + d->B : 0;
     pl->lse_off = kWsHeaderBytes;
     pl->o_off = align256(pl->lse_off + (size_t)pl->max_pieces * R * sizeof(float));
-    pl->bytes = pl->o_off + (size_t)pl->max_pieces * R * kDl * sizeof(float);
+    pl->bytes = pl->o_off + (size_t)pl->max_pieces * R * kDl * sizeof(__nv_bfloat16);
     return MLA_OK;
 }
 
@@ -148,7 +148,7 @@ int mla_decode(const void *q_lat, const void *q_pe, const void *kv_pages, const 
     char *ws = static_cast<char *>(workspace);
     p.err = reinterpret_cast<int32_t *>(ws);
     p.part_lse = reinterpret_cast<float *>(ws + pl.lse_off);
-    p.part_o = reinterpret_cast<float *>(ws + pl.o_off);
+    p.part_o = reinterpret_cast<__nv_bfloat16 *>(ws + pl.o_off);
     p.max_pieces = pl.max_pieces;
     p.B = dims->B;
     p.T = dims->T;

@@ -33,7 +33,9 @@ struct Problem {
     // sit next to each other, so the merge reads each row's parts as one
     // contiguous run (no large power-of-two stride that lands every part of a
     // row in the same cache slices)
-    float *part_o;                // [R, max_pieces, 512] normalised partial outputs
+    // bf16: the partials are half the bytes the attention kernel writes and the
+    // merge reads (2^-9 relative error each, far inside the parity tolerance)
+    __nv_bfloat16 *part_o;        // [R, max_pieces, 512] normalised partial outputs
     float *part_lse;              // [R, max_pieces]
     int64_t max_pieces;           // piece stride of the partials
     int32_t *err;                 // workspace error word {code, info}

@@ -32,10 +32,20 @@ struct Online {
     bool nan = false;
 };
 
+// Four consecutive dims of a part: fp32 (mla_merge_partials) or bf16 (the
+// decode's own split-KV partials).
+__device__ __forceinline__ float4 load4(const float *q) { return __ldg(reinterpret_cast<const float4 *>(q)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *q) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(q));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
 // parts first, first + step, ... < n of one unit: lse at l0[i*l_stride], the
-// lane's four dims at v0[i*v_stride] (float4 units)
-template <int kB>
-__device__ __forceinline__ void combine_parts(Online &st, const float *l0, int64_t l_stride, const float4 *v0,
+// lane's four dims at v0 + i*v_stride (elements)
+template <int kB, typename T>
+__device__ __forceinline__ void combine_parts(Online &st, const float *l0, int64_t l_stride, const T *v0,
                                               int64_t v_stride, int first, int step, int n) {
     for (int base = first; base < n; base += kB * step) {
         float l[kB];
@@ -46,7 +56,7 @@ __device__ __forceinline__ void combine_parts(Online &st, const float *l0, int64
             l[u] = -INFINITY;
             if (i < n) {
                 l[u] = __ldg(l0 + i * l_stride);
-                v[u] = __ldg(v0 + i * v_stride);
+                v[u] = load4(v0 + i * v_stride);
             }
         }
 #pragma unroll
@@ -109,13 +119,13 @@ struct MergeSmem {
 };
 
 // One unit, all eight warps of the CTA over its parts (many parts).
-__device__ __forceinline__ void merge_unit_cta(const float *o0, int64_t o_stride, const float *l0, int64_t l_stride,
+template <typename T>
+__device__ __forceinline__ void merge_unit_cta(const T *o0, int64_t o_stride, const float *l0, int64_t l_stride,
                                                int n, void *out, int64_t out_row, int quarter, int out_f32,
                                                float *lse_out, MergeSmem &sm) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     Online st;
-    combine_parts<kCtaBatch>(st, l0, l_stride, reinterpret_cast<const float4 *>(o0) + quarter * 32 + lane, o_stride / 4,
-                             warp, kWarps, n);
+    combine_parts<kCtaBatch>(st, l0, l_stride, o0 + quarter * 128 + lane * 4, o_stride, warp, kWarps, n);
     sm.acc[warp][lane] = st.acc;
     if (lane == 0) {
         sm.m[warp] = st.m;
@@ -144,13 +154,13 @@ __device__ __forceinline__ void merge_unit_cta(const float *o0, int64_t o_stride
 }
 
 // One unit per warp (few parts).
-__device__ __forceinline__ void merge_unit_warp(const float *o0, int64_t o_stride, const float *l0, int64_t l_stride,
+template <typename T>
+__device__ __forceinline__ void merge_unit_warp(const T *o0, int64_t o_stride, const float *l0, int64_t l_stride,
                                                 int n, void *out, int64_t out_row, int quarter, int out_f32,
                                                 float *lse_out) {
     const int lane = threadIdx.x & 31;
     Online st;
-    combine_parts<kBatch>(st, l0, l_stride, reinterpret_cast<const float4 *>(o0) + quarter * 32 + lane, o_stride / 4, 0,
-                          1, n);
+    combine_parts<kBatch>(st, l0, l_stride, o0 + quarter * 128 + lane * 4, o_stride, 0, 1, n);
     write_unit(st, out, out_row, quarter, lane, out_f32, lse_out);
 }
 
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, kCta ? 3 : 1) merge_internal_kernel(
     // schedule needs only ctx_lens); the partials are read after it is done.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the pieces of row r are contiguous: [r][piece][512]
-    const float *o0 = p.part_o + ((int64_t)r * p.max_pieces + piece_base) * kDl;
+    const __nv_bfloat16 *o0 = p.part_o + ((int64_t)r * p.max_pieces + piece_base) * kDl;
     const float *l0 = p.part_lse + (int64_t)r * p.max_pieces + piece_base;
     if (kCta)
         merge_unit_cta(o0, kDl, l0, 1, n_pieces, p.out, grow, quarter, p.out_f32, p.lse, sm);

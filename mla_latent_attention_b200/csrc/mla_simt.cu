@@ -173,8 +173,8 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(Problem p) {
                 if (tid == 0 && p.lse) p.lse[grow] = lse;
             } else {
                 int64_t prow = (int64_t)r * p.max_pieces + pc.piece;
-                p.part_o[prow * kDl + d0] = o0;
-                p.part_o[prow * kDl + d0 + 1] = o1;
+                p.part_o[prow * kDl + d0] = __float2bfloat16_rn(o0);
+                p.part_o[prow * kDl + d0 + 1] = __float2bfloat16_rn(o1);
                 if (tid == 0) p.part_lse[prow] = lse;
             }
         }

@@ -170,7 +170,7 @@ __device__ __forceinline__ bool aborted(Misc &ms) { return *reinterpret_cast<vol
 // runs out just before the phase completes cannot split the warp (the
 // .sync.aligned tensor-memory loads that follow need all of it).
 __device__ __forceinline__ bool waitb(const Problem &p, Misc &ms, uint64_t *bar, uint32_t parity) {
-    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, wait_limit(p)));
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, wait_limit(p), p.wait_limit != 0));
     if (!ok) cta_abort(p, ms);
     return ok;
 }
@@ -215,6 +215,7 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                          unsigned char *smem, Misc &ms, int slot) {
     using C = Cfg<kFp8>;
     const int lane = threadIdx.x & 31;
+    const uint64_t pol = ptx::policy_evict_first();  // the cache is read once: first out of L2
     uint32_t g = 0;            // tiles whose copies are all armed
     uint32_t cur_parts = 0;    // parts of tile g armed so far (a stop can come mid-tile)
     bool first_piece = true;
@@ -258,16 +259,16 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                 uint64_t *bar = &ms.part_full[stage][part];
                 if constexpr (kFp8) {
                     if (part == C::kRope) {
-                        ptx::tma_load_2d(st + C::kRopeOff + lane * 1024, map_b, bar, 512, y);
+                        ptx::tma_load_2d_hint(st + C::kRopeOff + lane * 1024, map_b, bar, 512, y, pol);
                     } else {
                         // page slot `lane` = 8-position groups 2*lane, 2*lane+1
-                        ptx::tma_load_5d(st + lane * 2 * C::kGroupStride, map_a, bar, 0, 0, 0, 0, pid);
+                        ptx::tma_load_5d_hint(st + lane * 2 * C::kGroupStride, map_a, bar, 0, 0, 0, 0, pid, pol);
                         if (!p.kv_scale_per_tensor)
-                            ptx::bulk_load(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
-                                           p.kv_scale + (int64_t)pid * kPage, 64, bar);
+                            ptx::bulk_load_hint(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
+                                                p.kv_scale + (int64_t)pid * kPage, 64, bar, pol);
                     }
                 } else {
-                    ptx::tma_load_2d(st + part * C::kChunkStride + lane * 2048, map_a, bar, 64 * part, y);
+                    ptx::tma_load_2d_hint(st + part * C::kChunkStride + lane * 2048, map_a, bar, 64 * part, y, pol);
                 }
             }
             cur_parts = 0;
@@ -375,7 +376,7 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
     // a phase that completes (or a limit that expires) while it waits.
     auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {
         int ok = 1;
-        if (lane == 0) ok = ptx::mbar_wait(bar, parity, wait_limit(p)) && !aborted(ms);
+        if (lane == 0) ok = ptx::mbar_wait(bar, parity, wait_limit(p), p.wait_limit != 0) && !aborted(ms);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) cta_abort(p, ms);
         return ok != 0;
@@ -450,11 +451,13 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
                 qp = 0;
                 s_ok = false;
             }
+            // no sleep between polls: a nanosleep here delayed the next issue
+            // by about a thousand cycles
             if (pick != 0) {
                 t_idle = ptx::cycles();
                 spins = 0;
-            } else if ((++spins & 3) == 0) {
-                __nanosleep(32);  // leave issue slots to the softmax warps of this scheduler
+            } else {
+                ++spins;
             }
             if (pick == 0 && (spins & 255) == 0) {
                 int expired = 0;
@@ -786,13 +789,18 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&ms.s_free[sb]);
 
+            // scores in log2 units; outside the visible range -inf (the
+            // per-row limits are read only for tiles that reach past one)
+            if (fast) {
+#pragma unroll
+                for (int c = 0; c < kRpt; ++c) s[c] *= factor;
+            } else {
+#pragma unroll
+                for (int c = 0; c < kRpt; ++c) s[c] = loaded && pos < ms.col_lim[cb + c] ? s[c] * factor : -INFINITY;
+            }
             bool exceed = false;
 #pragma unroll
-            for (int c = 0; c < kRpt; ++c) {
-                const bool valid = fast || (loaded && pos < ms.col_lim[cb + c]);
-                s[c] = valid ? s[c] * factor : -INFINITY;       // score, log2 units
-                exceed |= s[c] > m2c[c] + kx;
-            }
+            for (int c = 0; c < kRpt; ++c) exceed |= s[c] > m2c[c] + kx;
             // Optimistic stabiliser: every warp writes its weights with the
             // current stabiliser and flags the tile if one of them would be too
             // large; the tile's fate is read once every warp has written it.
@@ -885,7 +893,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         for (int c = 0; c < kRpt; ++c) {
             const float l = ms.red[h][0][c] + ms.red[h][1][c] + ms.red[h][2][c] + ms.red[h][3][c];
             const bool bad = piece_bad || ms.col_bad[cb + c];
-            inv_l[c] = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+            inv_l[c] = bad ? NAN : (l > 0.f ? __frcp_rn(l) : 0.f);
             // ln sum_j exp(score_j) = (m2c + log2 l) * ln 2
             if (c == hst) row_lse = bad ? NAN : (l > 0.f ? (m2c[c] + __log2f(l)) * kLn2 : -INFINITY);
         }
@@ -895,7 +903,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         // the next piece), and the group's first thread stores the box with a
         // tensor store; the maps clip rows past the sequence's R.
         const int nrows = min(kRpt, rows_here - cb);
-        const bool f32_box = !pc.single || p.out_f32;
+        const bool f32_box = pc.single && p.out_f32;   // partials are bf16
         constexpr int kBoxBytes = kRpt * 128 * 4;
 #pragma unroll 1
         for (int m = 0; m < 4; ++m) {
@@ -1061,7 +1069,7 @@ bool make_fp8_latent_map(CUtensorMap *map, const void *base, int num_pages) {
 
 // Output views for the epilogue's tensor stores, boxes of 128 dims x 16 rows
 // (one softmax row group): out as [B][R][512] (bf16 or fp32), the partials
-// as [R][pieces][512] fp32.
+// as [R][pieces][512] bf16.
 bool make_out_maps(CUtensorMap *mo, CUtensorMap *mp, const Problem &p) {
     auto encode = get_encode_fn();
     if (!encode) return false;
@@ -1081,9 +1089,9 @@ bool make_out_maps(CUtensorMap *mo, CUtensorMap *mp, const Problem &p) {
         return true;
     }
     const cuuint64_t dims[3] = {(cuuint64_t)kDl, (cuuint64_t)p.max_pieces, (cuuint64_t)p.R};
-    const cuuint64_t strides[2] = {(cuuint64_t)kDl * 4, (cuuint64_t)p.max_pieces * kDl * 4};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDl * 2, (cuuint64_t)p.max_pieces * kDl * 2};
     const cuuint32_t box[3] = {128, 1, (cuuint32_t)kRpt};
-    return encode(mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.part_o, dims, strides, box, estr,
+    return encode(mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.part_o, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -69,11 +69,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_cycles` SM cycles and returns false, so that no wait can hang.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_cycles) {
-    if (mbar_try_wait(bar, parity)) return true;
+// try_wait may suspend the thread in hardware for a while before it returns,
+// so the limit is checked between hardware waits; with `poll` the wait polls
+// the barrier without suspending instead, and the limit holds to within a
+// few hundred cycles (a short limit set by the caller).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_cycles, bool poll = false) {
+    if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = cycles();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (poll ? mbar_test(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (cycles() - t0 > limit_cycles) return false;
     }
 }
@@ -87,13 +91,35 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// 5-D tensor tile load (the FP8 page view: bytes x rows x chunks x halves x pages).
-__device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2,
-                                            int c3, int c4) {
+// L2 cache policy that makes the lines a copy brings in the first to be
+// evicted: the KV cache is streamed once per decode, and with the default
+// policy it would push the kernel's code and the small inputs out of L2
+// between launches.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 2-D tensor tile load with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                                 uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], "
-        "[%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+        "%4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+        : "memory");
+}
+
+// 5-D tensor tile load (the FP8 page view: bytes x rows x chunks x halves x
+// pages) with an L2 cache policy.
+__device__ __forceinline__ void tma_load_5d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                                 int c2, int c3, int c4, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+        "%4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+        "l"(pol)
         : "memory");
 }
 
@@ -111,6 +137,16 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Plain bulk copy global -> shared with an L2 cache policy.
+__device__ __forceinline__ void bulk_load_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                               uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
 }
 
 // Plain bulk copy global -> shared (16-byte aligned addresses, size multiple of 16).
