@@ -76,8 +76,10 @@ int make_plan(const mla_dims *d, Plan *pl) {
     } else {
         const int ctas_per_sm = pl->kernel == MLA_KERNEL_SIMT ? 2 : 1;
         slots = (int64_t)sms * ctas_per_sm / pl->n_groups;
-        // no range shorter than 8 pages (one 128-position tile) on average
-        const int64_t page_bound = ((int64_t)d->B * d->max_pages_per_seq + 7) / 8;
+        // no range shorter than 16 pages (two 128-position tiles) on average:
+        // a CTA with less work spends most of its time in its fixed costs, and
+        // a history that fits one range needs no merge kernel at all
+        const int64_t page_bound = ((int64_t)d->B * d->max_pages_per_seq + 15) / 16;
         if (slots > page_bound) slots = page_bound;
         if (slots < 1) slots = 1;
     }

@@ -70,6 +70,7 @@ constexpr int kSoftmaxWarps = 4 * kRowGroups;       // x 4 TMEM lane quadrants
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kThreads = 64 + kSoftmaxThreads;      // warp 0 TMA, warp 1 MMA, warps 2.. softmax
 constexpr int kRpt = kN / kRowGroups;               // query rows per softmax thread
+static_assert(kRpt == 16, "the row reductions and the paired score loads take 16 rows per thread");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimit = 4000000000ull;  // SM cycles: about two seconds
 
@@ -151,7 +152,8 @@ struct Misc {
     int col_bad[kN];
     float qscale;
     float amax[kSoftmaxWarps];
-    float red[kRowGroups][4][kRpt];  // [row group][warp][row]
+    __align__(16) float red[kRowGroups][4][kRpt];  // [row group][warp][row]
+    float m2c[kN];            // per row: the stabiliser (minus C) at the end of a piece
 };
 
 template <bool kFp8>
@@ -205,6 +207,28 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// Reduces 16 per-lane values x[r] + off (one per row) over the warp's 32
+// lanes by halving exchanges (8 + 4 + 2 + 1 + 1 shuffles instead of 16 x 5):
+// the result for row r is returned in lanes 2r and 2r + 1.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_rows16(const float (&x)[16], float off = 0.f) {
+    const int lane = threadIdx.x & 31;
+    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+    float v8[8], v4[4], v2[2];
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        v8[j] = op((b4 ? x[8 + j] : x[j]) + off, __shfl_xor_sync(0xffffffffu, (b4 ? x[j] : x[8 + j]) + off, 16));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        v4[j] = op(b3 ? v8[4 + j] : v8[j], __shfl_xor_sync(0xffffffffu, b3 ? v8[j] : v8[4 + j], 8));
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+        v2[j] = op(b2 ? v4[2 + j] : v4[j], __shfl_xor_sync(0xffffffffu, b2 ? v4[j] : v4[2 + j], 4));
+    const float v1 = op(b1 ? v2[1] : v2[0], __shfl_xor_sync(0xffffffffu, b1 ? v2[0] : v2[1], 2));
+    return op(v1, __shfl_xor_sync(0xffffffffu, v1, 1));
 }
 
 // ---------------------------------------------------------------------------
@@ -513,7 +537,9 @@ __device__ bool stage_query(const Problem &p, unsigned char *smem, Misc &ms, int
         constexpr int kUnits = kN * 36;
         constexpr int kPer = (kUnits + kSoftmaxThreads - 1) / kSoftmaxThreads;  // 7
         uint4 v[kPer][2];
-        float amax = 0.f;
+        // largest |q| from the bf16 bit patterns: with the sign cleared, a
+        // bf16 magnitude orders like its bits, two per 32-bit word
+        uint32_t mbits = 0;
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int u = st + j * kSoftmaxThreads;
@@ -527,14 +553,14 @@ __device__ bool stage_query(const Problem &p, unsigned char *smem, Misc &ms, int
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v[j][h]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(b2[e]);
-                    amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-                }
+                mbits = __vmaxu2(mbits, v[j][h].x & 0x7FFF7FFFu);
+                mbits = __vmaxu2(mbits, v[j][h].y & 0x7FFF7FFFu);
+                mbits = __vmaxu2(mbits, v[j][h].z & 0x7FFF7FFFu);
+                mbits = __vmaxu2(mbits, v[j][h].w & 0x7FFF7FFFu);
             }
         }
+        mbits = max(mbits & 0xFFFFu, mbits >> 16);
+        float amax = __uint_as_float(mbits << 16);
         amax = warp_max(amax);
         if ((threadIdx.x & 31) == 0) ms.amax[(threadIdx.x >> 5) - 2] = amax;
         if (!gsync(p, ms)) return false;   // also: every raw read is done
@@ -672,6 +698,9 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         const int rows_here = min(kN, p.R - r0);
         int min_lim = INT_MAX;  // over this row group's real rows
         for (int c = cb; c < min(cb + kRpt, rows_here); ++c) min_lim = min(min_lim, ms.col_lim[c]);
+        uint32_t bad_rows = 0;  // bit c: row cb + c is invalid (its results are NaN)
+#pragma unroll
+        for (int c = 0; c < kRpt; ++c) bad_rows |= ms.col_bad[cb + c] ? 1u << c : 0u;
 
         if (nt == 0) {  // nothing to read: write the empty (or invalid) result
             for (int e = st; e < rows_here * kDl; e += kSoftmaxThreads) {
@@ -834,18 +863,27 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             // stabiliser of the rows whose weights overflowed to DELTA above
             // their new maximum, rescale what came before, rewrite P.  The
             // value MMAs of this tile wait for it (p_redo).
-#pragma unroll
-            for (int c = 0; c < kRpt; ++c) {
-                const float cm = warp_max(s[c] + lkvs);
-                if (lane == 0) ms.red[h][w4][c] = cm;
+            {
+                const float v = warp_reduce_rows16<true>(s, lkvs);   // max over lanes of score + lkvs
+                if ((lane & 1) == 0) ms.red[h][w4][lane >> 1] = v;
             }
             if (!all_sync(p, ms)) return;
+            float cmax[kRpt];
+#pragma unroll
+            for (int c4 = 0; c4 < kRpt / 4; ++c4) {
+                float4 a = reinterpret_cast<const float4 *>(ms.red[h][0])[c4];
+#pragma unroll
+                for (int w = 1; w < 4; ++w) {
+                    const float4 t = reinterpret_cast<const float4 *>(ms.red[h][w])[c4];
+                    a.x = fmaxf(a.x, t.x); a.y = fmaxf(a.y, t.y); a.z = fmaxf(a.z, t.z); a.w = fmaxf(a.w, t.w);
+                }
+                cmax[4 * c4] = a.x; cmax[4 * c4 + 1] = a.y; cmax[4 * c4 + 2] = a.z; cmax[4 * c4 + 3] = a.w;
+            }
             float alpha[kRpt];
             bool moved = false;
 #pragma unroll
             for (int c = 0; c < kRpt; ++c) {
-                const float cm = fmaxf(fmaxf(ms.red[h][0][c], ms.red[h][1][c]),
-                                       fmaxf(ms.red[h][2][c], ms.red[h][3][c]));
+                const float cm = cmax[c];
                 const float old = m2c[c] + C::kC;
                 const float mn = cm > old + C::kTau ? cm + C::kDelta : old;
                 alpha[c] = mn == old ? 1.f : ptx::ex2(old - mn);
@@ -876,26 +914,45 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         g = g0 + nt;
 
         // ---- epilogue: row sums, normalised output, log-sum-exp
+        if (piece_bad) bad_rows = 0xFFFFu;
         // the last value MMAs done (a commit covers every earlier MMA too)
         if (!waitb(p, ms, &ms.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) return;
         ptx::tc_fence_after();
+        // the warp's row sums over its 32 lanes, one row per lane pair
+        {
+            const float v = warp_reduce_rows16<false>(lsum);
+            if ((lane & 1) == 0) ms.red[h][w4][lane >> 1] = v;
+        }
+        // the group's stabilisers, for the rows' log-sum-exps
+        if (hst == 0) {
 #pragma unroll
-        for (int c = 0; c < kRpt; ++c) {
-            const float v = warp_sum(lsum[c]);
-            if (lane == 0) ms.red[h][w4][c] = v;
+            for (int c = 0; c < kRpt; ++c) ms.m2c[cb + c] = m2c[c];
         }
         if (!hsync(p, ms)) return;
-        // every thread forms the sums of its own rows; thread hst < kRpt of the
-        // group also forms row cb + hst's log-sum-exp
+        // every thread forms the sums of its own rows (vector loads of the four
+        // warps' parts); thread hst < kRpt of the group also forms row cb +
+        // hst's log-sum-exp
         float inv_l[kRpt];
-        float row_lse = 0.f;
 #pragma unroll
-        for (int c = 0; c < kRpt; ++c) {
-            const float l = ms.red[h][0][c] + ms.red[h][1][c] + ms.red[h][2][c] + ms.red[h][3][c];
-            const bool bad = piece_bad || ms.col_bad[cb + c];
-            inv_l[c] = bad ? NAN : (l > 0.f ? __frcp_rn(l) : 0.f);
+        for (int c4 = 0; c4 < kRpt / 4; ++c4) {
+            float4 l = reinterpret_cast<const float4 *>(ms.red[h][0])[c4];
+#pragma unroll
+            for (int w = 1; w < 4; ++w) {
+                const float4 t = reinterpret_cast<const float4 *>(ms.red[h][w])[c4];
+                l.x += t.x; l.y += t.y; l.z += t.z; l.w += t.w;
+            }
+            const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int c = 4 * c4 + e;
+                inv_l[c] = (bad_rows >> c) & 1u ? NAN : (lv[e] > 0.f ? __fdividef(1.f, lv[e]) : 0.f);
+            }
+        }
+        float row_lse = 0.f;
+        if (hst < kRpt) {
+            const float l = ms.red[h][0][hst] + ms.red[h][1][hst] + ms.red[h][2][hst] + ms.red[h][3][hst];
             // ln sum_j exp(score_j) = (m2c + log2 l) * ln 2
-            if (c == hst) row_lse = bad ? NAN : (l > 0.f ? (m2c[c] + __log2f(l)) * kLn2 : -INFINITY);
+            row_lse = (bad_rows >> hst) & 1u ? NAN : (l > 0.f ? (ms.m2c[cb + hst] + __log2f(l)) * kLn2 : -INFINITY);
         }
         // O goes out one 128-dim block at a time, each row group on its own:
         // the group's threads write their dims of its 16 rows into a [16][128]

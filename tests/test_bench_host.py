@@ -172,3 +172,12 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert len(lines) == 1, r.stdout
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["value"] > 0
+
+
+def test_split_step_divides_the_timed_layer():
+    """The per-kernel times are the timed per-layer time divided in the
+    proportion the event nodes measured, so they add up to the step."""
+    att, mer = bench.split_step(60.0, 66.0, 11.0)
+    assert abs(att + mer - 60.0) < 1e-9
+    assert abs(att / mer - 6.0) < 1e-9
+    assert bench.split_step(10.0, 0.0, 0.0) == (10.0, 0.0)
