@@ -26,13 +26,15 @@
 //     adds the two halves of O^T.  V is read as stored, never dequantised.
 // bf16 caches use kind::f16 MMAs with N = 48 and bf16 P.
 //
-// Warp roles (448 threads): warp 0 issues TMA page loads, warp 1 issues the
-// MMAs -- each group as soon as its operands are ready -- and owns tensor
-// memory, warps 2-13 run the online softmax and the epilogue.  Thread
+// Warp roles (480 threads): warp 0 issues TMA page loads, warp 1 issues the
+// score MMAs and owns tensor memory, warp 14 issues the value MMAs, warps
+// 2-13 run the online softmax and the epilogue.  Thread
 // (warp w, lane l) owns tile position / TMEM lane 32*(w%4) + l; the softmax
 // warps form three groups of four (one per TMEM lane quadrant), each group
-// taking 16 of the 48 query rows.  (Fourteen warps leave 128 registers per
-// thread; sixteen softmax warps of 12 rows would leave 96 and spill.)
+// taking 16 of the 48 query rows.  (Fifteen warps get 128 registers per
+// thread: the register file is split over four sub-partitions, each holding
+// four of the warps at most.  Sixteen softmax warps of 12 rows would leave 96
+// and spill.)
 //
 // Softmax stabiliser: per query row a running bound m2 on the log2 weight
 // u = s*log2(e)*scale (+ log2 of the token's value scale for FP8), shared by
@@ -45,8 +47,8 @@
 // with the current bound and flags the tile if one would exceed it; once
 // every warp has written the tile (the same barrier the value MMAs wait on),
 // a flagged tile takes a slow path in which all softmax warps agree on the
-// new bounds, rescale, and rewrite the weights, and the MMA warp issues that
-// tile's value MMAs only after the rewrite.  The first tile of every piece is
+// new bounds, rescale, and rewrite the weights, and the value MMAs of that
+// tile are issued only after the rewrite.  The first tile of every piece is
 // flagged (no bound yet); later ones almost never are.
 
 // Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA
@@ -68,7 +70,8 @@ constexpr int kTilePages = kTileM / kPage;
 constexpr int kRowGroups = 3;                       // softmax warp sets, one per 16 of the 48 rows
 constexpr int kSoftmaxWarps = 4 * kRowGroups;       // x 4 TMEM lane quadrants
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
-constexpr int kThreads = 64 + kSoftmaxThreads;      // warp 0 TMA, warp 1 MMA, warps 2.. softmax
+constexpr int kValueWarp = 2 + kSoftmaxWarps;      // warp 0 TMA, warp 1 score MMAs, 2..13 softmax
+constexpr int kThreads = 32 * (kValueWarp + 1);     // and the value MMAs' warp
 constexpr int kRpt = kN / kRowGroups;               // query rows per softmax thread
 static_assert(kRpt == 16, "the row reductions and the paired score loads take 16 rows per thread");
 constexpr uint32_t kTmemCols = 512;
@@ -203,12 +206,6 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
 // Reduces 16 per-lane values x[r] + off (one per row) over the warp's 32
 // lanes by halving exchanges (8 + 4 + 2 + 1 + 1 shuffles instead of 16 x 5):
 // the result for row r is returned in lanes 2r and 2r + 1.
@@ -314,23 +311,48 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
 }
 
 // ---------------------------------------------------------------------------
-// warp 1: MMA issuer
+// warps 1 and 14: MMA issuers
 // ---------------------------------------------------------------------------
+// The score MMAs of a tile and the value MMAs of the tile before it are
+// issued by two warps.  Issuing a group of MMAs blocks the issuing thread
+// until most of the group has run, about a thousand cycles; with one issuer
+// the value MMAs of tile k, whose completion frees the KV stage that tile
+// k + 2 is copied into, waited behind that block whenever the scores of tile
+// k + 1 had just been issued.  With two, each issuer waits only for what its
+// own MMAs read, and the tensor pipe takes the two groups as they come.
+//
+// A commit tracks the MMAs of its own thread.  The KV stage part that both
+// groups read is freed by the value group's commit alone: by then the scores
+// of that tile have been read by the softmax, so their MMAs are done.
+
+// Waits are made by lane 0 and broadcast, so the warp never diverges on a
+// phase that completes (or a limit that expires) while it waits.
+__device__ __forceinline__ bool issuer_wait(const Problem &p, Misc &ms, uint64_t *bar, uint32_t parity) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = ptx::mbar_wait(bar, parity, wait_limit(p), p.wait_limit != 0) && !aborted(ms);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) cta_abort(p, ms);
+    return ok != 0;
+}
+
+// every MMA this thread issued has completed before tensor memory is released
+__device__ __forceinline__ void issuer_drain(Misc &ms) {
+    if ((threadIdx.x & 31) == 0) ptx::mma_commit(&ms.drain);
+    __syncwarp();
+    ptx::mbar_wait(&ms.drain, 0, kWaitLimit);
+}
+
+// warp 1: score MMAs S^T = K Q^T of every tile, once its parts have landed
+// and the score buffer is free.
 template <bool kFp8>
-__device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int slot) {
+__device__ void score_issuer(const Problem &p, unsigned char *smem, Misc &ms, int slot) {
     using C = Cfg<kFp8>;
     const int lane = threadIdx.x & 31;
     const uint32_t tmem = ms.tmem_base;
     const uint32_t kv0 = ptx::smem_u32(smem + C::kKvOff);
     const uint32_t q0 = ptx::smem_u32(smem + C::kQOff);
-    const uint32_t p0 = ptx::smem_u32(smem + C::kPOff);
     constexpr uint32_t idesc_qk = kFp8 ? ptx::instr_desc(0, 0, 0, 0, kTileM, C::kNMma)
                                        : ptx::instr_desc(1, 1, 0, 0, kTileM, C::kNMma);
-    constexpr uint32_t idesc_pv = kFp8 ? ptx::instr_desc(0, 0, 1, 1, kTileM, C::kNMma)
-                                       : ptx::instr_desc(1, 1, 1, 1, kTileM, C::kNMma);
-    uint32_t g = 0, pi = 0;
-    uint32_t redo_n = 0;       // rewrites of flagged tiles' weights consumed (lane 0)
-
     // Shared-memory descriptors are built once; an MMA then only adds the
     // byte offset of its operands (>> 4) to the start-address field.
     constexpr uint64_t kStageStep = (uint64_t)(C::kStageBytes >> 4);
@@ -338,9 +360,6 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
     const uint64_t dq_q = ptx::smem_desc(q0, 16, 1024, ptx::kSwizzle128B);
     const uint64_t dr_kv = ptx::smem_desc(kv0 + C::kRopeOff, 16, 512, ptx::kSwizzle64B);  // FP8 RoPE
     const uint64_t dr_q = ptx::smem_desc(q0 + C::kQRopeOff, 16, 512, ptx::kSwizzle64B);
-    // V^T, MN-major: 128-B atoms along the dims C::kChunkStride apart, 8-position groups along K
-    const uint64_t dv_kv = ptx::smem_desc(kv0, C::kChunkStride, C::kGroupStride, ptx::kSwizzle128B);
-    const uint64_t dv_p = ptx::smem_desc(p0, 128, 2048, ptx::kSwizzleNone);       // P^T, MN-major
 
     // Score MMAs reading one part of the tile (accumulate from the second MMA of the tile on).
     auto issue_qk_part = [&](uint32_t gg, int part, bool first) {
@@ -371,6 +390,49 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
         }
     };
 
+    uint32_t g = 0, pi = 0;
+    for_each_piece(p, slot, [&](const Piece &pc) {
+        const int nt = ntiles_of(pc);
+        if (nt == 0 || aborted(ms)) return;
+        if (!issuer_wait(p, ms, &ms.q_ready, pi & 1)) return;
+        for (int k = 0; k < nt; ++k) {
+            const uint32_t gq = g + k;
+            const int stage = gq % C::kStages;
+            if (!issuer_wait(p, ms, &ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1)) return;
+            for (int q = 0; q < C::kParts; ++q)
+                if (!issuer_wait(p, ms, &ms.part_full[stage][q == 0 ? C::kRope : q - 1], (gq / C::kStages) & 1))
+                    return;
+            ptx::tc_fence_after();
+            if (lane == 0) {
+#pragma unroll
+                for (int q = 0; q < C::kParts; ++q) issue_qk_part(gq, q == 0 ? C::kRope : q - 1, q == 0);
+                ptx::mma_commit(&ms.s_full[gq % C::kSBufs]);
+                ptx::mma_commit(&ms.part_empty[stage][C::kRope]);  // RoPE is read by scores only
+            }
+            __syncwarp();
+        }
+        g += nt;
+        ++pi;
+    });
+    issuer_drain(ms);
+}
+
+// warp 14: value MMAs O^T += V^T P^T of every tile, once all softmax warps
+// have written its weights (and, for a flagged tile, rewritten them).
+template <bool kFp8>
+__device__ void value_issuer(const Problem &p, unsigned char *smem, Misc &ms, int slot) {
+    using C = Cfg<kFp8>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t tmem = ms.tmem_base;
+    const uint32_t kv0 = ptx::smem_u32(smem + C::kKvOff);
+    const uint32_t p0 = ptx::smem_u32(smem + C::kPOff);
+    constexpr uint32_t idesc_pv = kFp8 ? ptx::instr_desc(0, 0, 1, 1, kTileM, C::kNMma)
+                                       : ptx::instr_desc(1, 1, 1, 1, kTileM, C::kNMma);
+    constexpr uint64_t kStageStep = (uint64_t)(C::kStageBytes >> 4);
+    // V^T, MN-major: 128-B atoms along the dims C::kChunkStride apart, 8-position groups along K
+    const uint64_t dv_kv = ptx::smem_desc(kv0, C::kChunkStride, C::kGroupStride, ptx::kSwizzle128B);
+    const uint64_t dv_p = ptx::smem_desc(p0, 128, 2048, ptx::kSwizzleNone);       // P^T, MN-major
+
     // Value MMAs; each 128-dim block frees its value chunk(s) of the stage as it completes.
     auto issue_pv = [&](uint32_t gg, bool first) {
         const int stage = gg % C::kStages;
@@ -396,109 +458,35 @@ __device__ void mma_issuer(const Problem &p, unsigned char *smem, Misc &ms, int 
         if constexpr (kFp8) ptx::mma_commit(&ms.part_empty[stage][0]);
     };
 
-    // Waits are made by lane 0 and broadcast, so the warp never diverges on
-    // a phase that completes (or a limit that expires) while it waits.
-    auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {
-        int ok = 1;
-        if (lane == 0) ok = ptx::mbar_wait(bar, parity, wait_limit(p), p.wait_limit != 0) && !aborted(ms);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) cta_abort(p, ms);
-        return ok != 0;
-    };
-
-    // Two groups per tile k: the scores of tile k (all its parts landed and
-    // the score buffer free) and the values of tile k - 1 (its weights
-    // written).  Lane 0 polls both and the warp issues whichever is ready
-    // first; the values go first when both are, since they free the stage
-    // that the next copy waits for.
+    uint32_t g = 0, pi = 0;
+    uint32_t redo_n = 0;       // rewrites of flagged tiles' weights consumed
     for_each_piece(p, slot, [&](const Piece &pc) {
         const int nt = ntiles_of(pc);
         if (nt == 0 || aborted(ms)) return;
-        const uint32_t g0 = g;
-        if (!wait1(&ms.q_ready, pi & 1)) return;
-        int nq = 0, nv = 0;        // score / value groups issued
-        int qp = 0;                // parts of tile nq seen landed
-        bool s_ok = false, o_ok = false, p_ok = false;
-        int redo_state = 0;        // tile nv: 0 not read, 1 weights final, 2 being rewritten
-        uint64_t t_idle = ptx::cycles();
-        uint32_t spins = 0;
-        while (nv < nt) {
-            // lane 0 decides; 1 = values, 2 = scores, 0 = nothing ready yet
-            int pick = 0;
+        for (int k = 0; k < nt; ++k) {
+            const uint32_t gp = g + k;
+            // the epilogue of the previous piece has read O
+            if (k == 0 && !issuer_wait(p, ms, &ms.o_free, (pi & 1) ^ 1)) return;
+            if (!issuer_wait(p, ms, &ms.p_full[gp & 1], (gp >> 1) & 1)) return;
+            // the flag was written before the last arrival on p_full
+            int redo = 0;
+            if (lane == 0) redo = *reinterpret_cast<volatile uint32_t *>(&ms.redo[gp & 1]) == gp + 1;
+            redo = __shfl_sync(0xffffffffu, redo, 0);
+            if (redo) {
+                if (!issuer_wait(p, ms, &ms.p_redo, redo_n & 1)) return;
+                ++redo_n;
+            }
+            ptx::tc_fence_after();
             if (lane == 0) {
-                if (nv < nq) {
-                    const uint32_t gp = g0 + nv;
-                    if (nv == 0 && !o_ok) o_ok = ptx::mbar_test(&ms.o_free, (pi & 1) ^ 1);
-                    if ((nv > 0 || o_ok) && !p_ok) p_ok = ptx::mbar_test(&ms.p_full[gp & 1], (gp >> 1) & 1);
-                    if (p_ok) {
-                        // the flag was written before the last arrival on p_full
-                        if (redo_state == 0)
-                            redo_state = *reinterpret_cast<volatile uint32_t *>(&ms.redo[gp & 1]) == gp + 1 ? 2 : 1;
-                        if (redo_state == 1 || ptx::mbar_test(&ms.p_redo, redo_n & 1)) pick = 1;
-                    }
-                }
-                if (pick == 0 && nq < nt && nq <= nv + 1) {
-                    const uint32_t gq = g0 + nq;
-                    const int stage = gq % C::kStages;
-                    if (!s_ok) s_ok = ptx::mbar_test(&ms.s_free[gq % C::kSBufs], ((gq / C::kSBufs) & 1) ^ 1);
-                    while (s_ok && qp < C::kParts &&
-                           ptx::mbar_test(&ms.part_full[stage][qp == 0 ? C::kRope : qp - 1], (gq / C::kStages) & 1))
-                        ++qp;
-                    if (s_ok && qp == C::kParts) pick = 2;
-                }
+                issue_pv(gp, k == 0);
+                ptx::mma_commit(&ms.pv_done[gp & 1]);
             }
-            pick = __shfl_sync(0xffffffffu, pick, 0);
-            if (pick == 1) {
-                const uint32_t gp = g0 + nv;
-                ptx::tc_fence_after();
-                if (lane == 0) {
-                    issue_pv(gp, nv == 0);
-                    ptx::mma_commit(&ms.pv_done[gp & 1]);
-                    if (redo_state == 2) ++redo_n;
-                    p_ok = false;
-                    redo_state = 0;
-                }
-                __syncwarp();
-                ++nv;
-            } else if (pick == 2) {
-                const uint32_t gq = g0 + nq;
-                const int stage = gq % C::kStages;
-                ptx::tc_fence_after();
-                if (lane == 0) {
-#pragma unroll
-                    for (int q = 0; q < C::kParts; ++q) issue_qk_part(gq, q == 0 ? C::kRope : q - 1, q == 0);
-                    ptx::mma_commit(&ms.s_full[gq % C::kSBufs]);
-                    ptx::mma_commit(&ms.part_empty[stage][C::kRope]);  // RoPE is read by scores only
-                }
-                __syncwarp();
-                ++nq;
-                qp = 0;
-                s_ok = false;
-            }
-            // no sleep between polls: a nanosleep here delayed the next issue
-            // by about a thousand cycles
-            if (pick != 0) {
-                t_idle = ptx::cycles();
-                spins = 0;
-            } else {
-                ++spins;
-            }
-            if (pick == 0 && (spins & 255) == 0) {
-                int expired = 0;
-                if (lane == 0) expired = (ptx::cycles() - t_idle > wait_limit(p)) || aborted(ms);
-                if (__shfl_sync(0xffffffffu, expired, 0)) {
-                    cta_abort(p, ms);
-                    return;
-                }
-            }
+            __syncwarp();
         }
-        g = g0 + nt;
+        g += nt;
         ++pi;
     });
-    // every MMA issued has completed before tensor memory is released
-    if (lane == 0) ptx::mma_commit(&ms.drain);
-    __syncwarp();
-    ptx::mbar_wait(&ms.drain, 0, kWaitLimit);
+    issuer_drain(ms);
 }
 
 // ---------------------------------------------------------------------------
@@ -733,18 +721,21 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         const uint32_t g0 = g;
 
         // This thread's entries of the tile's weight operand P: e = ex2(s - m2c)
-        // for its kRpt rows (times the token's value scale for FP8), written to
-        // P buffer gg & 1 in the layout the value MMA reads.  With add_sums the
-        // weights also enter the row sums.
-        auto store_p = [&](const float (&sc)[kRpt], float kvs, bool add_sums, uint32_t gg) {
-            unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
+        // for its kRpt rows (times the token's value scale for FP8), as the
+        // 32-bit words of the layout the value MMA reads (make_p), then written
+        // to P buffer gg & 1 (put_p).  With add_sums the weights also enter the
+        // row sums.  The conversions need no buffer, so they run before the
+        // wait for one.
+        constexpr int kPW = kFp8 ? kRpt / 4 : kRpt / 2;   // words per operand (hi, lo)
+        auto make_p = [&](const float (&sc)[kRpt], float kvs, bool add_sums, uint32_t (&hw)[kPW],
+                          uint32_t (&lw)[kPW]) {
             if constexpr (kFp8) {
                 // P = hi + lo, two e4m3 operands; word w packs rows 4w..4w+3 of this
                 // thread's rows.  Pairs go through f16x2: p16 = f16(P) (relative error 2^-12,
                 // far below lo's 2^-9), hi = e4m3(p16), and p16 - hi is exact in
                 // f16, so lo = e4m3(p16 - hi).
 #pragma unroll
-                for (int w = 0; w < kRpt / 4; ++w) {
+                for (int w = 0; w < kPW; ++w) {
                     uint32_t hp[2], lp[2];
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
@@ -758,28 +749,39 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                         hp[q] = ptx::e4m3x2_from_f16x2(p16);
                         lp[q] = ptx::e4m3x2_from_f16x2(ptx::sub_f16x2(p16, ptx::f16x2_from_e4m3x2(hp[q])));
                     }
-                    // P^T is [16-row groups of 16 B] x 128 positions; each four of this
-                    // thread's rows lie in one group
-                    const int row0 = cb + 4 * w;
-                    const int off = (row0 >> 4) * 2048 + i * 16 + (row0 & 15);
-                    *reinterpret_cast<uint32_t *>(pb + off) = hp[0] | (hp[1] << 16);
-                    *reinterpret_cast<uint32_t *>(pb + C::kPLoOff + off) = lp[0] | (lp[1] << 16);
+                    hw[w] = hp[0] | (hp[1] << 16);
+                    lw[w] = lp[0] | (lp[1] << 16);
                 }
             } else {
-                // bf16 P^T: [8-row groups of 16 B] x 128 positions, two rows per word
+                // bf16: word w packs rows 2w, 2w+1
 #pragma unroll
-                for (int w = 0; w < kRpt / 2; ++w) {
+                for (int w = 0; w < kPW; ++w) {
                     const int c0 = 2 * w;
                     const float e0 = ptx::ex2(sc[c0] - m2c[c0]), e1 = ptx::ex2(sc[c0 + 1] - m2c[c0 + 1]);
                     if (add_sums) {
                         lsum[c0] += e0;
                         lsum[c0 + 1] += e1;
                     }
-                    const int row0 = cb + c0;
                     __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
-                    *reinterpret_cast<uint32_t *>(pb + (row0 >> 3) * 2048 + i * 16 + 2 * (row0 & 7)) =
-                        *reinterpret_cast<uint32_t *>(&b2);
+                    hw[w] = *reinterpret_cast<uint32_t *>(&b2);
+                    lw[w] = 0u;
                 }
+            }
+        };
+        auto put_p = [&](const uint32_t (&hw)[kPW], const uint32_t (&lw)[kPW], uint32_t gg) {
+            unsigned char *pb = smem + C::kPOff + (gg & 1) * C::kPBytes;
+            if constexpr (kFp8) {
+                // P^T is [16-row groups of 16 B] x 128 positions: this thread's 16 rows
+                // (cb is a multiple of 16) are one 16-B entry of hi and one of lo, so a
+                // warp writes 512 contiguous bytes per store
+                const int off = (cb >> 4) * 2048 + i * 16;
+                *reinterpret_cast<uint4 *>(pb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(pb + C::kPLoOff + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            } else {
+                // bf16 P^T: [8-row groups of 16 B] x 128 positions: two entries
+                const int off = (cb >> 3) * 2048 + i * 16;
+                *reinterpret_cast<uint4 *>(pb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(pb + off + 2048) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
@@ -827,13 +829,17 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
 #pragma unroll
                 for (int c = 0; c < kRpt; ++c) s[c] = loaded && pos < ms.col_lim[cb + c] ? s[c] * factor : -INFINITY;
             }
-            bool exceed = false;
+            float dmax = s[0] - m2c[0];
 #pragma unroll
-            for (int c = 0; c < kRpt; ++c) exceed |= s[c] > m2c[c] + kx;
+            for (int c = 1; c < kRpt; ++c) dmax = fmaxf(dmax, s[c] - m2c[c]);
+            const bool exceed = dmax > kx;
             // Optimistic stabiliser: every warp writes its weights with the
             // current stabiliser and flags the tile if one of them would be too
             // large; the tile's fate is read once every warp has written it.
             const bool wex = __any_sync(0xffffffffu, exceed);
+            uint32_t hw[kPW], lw[kPW];
+            // a flagged warp's weights are rewritten below, and its sums added then
+            make_p(s, kvs, !wex, hw, lw);
             // P buffer gg & 1 is free once the value MMAs of tile gg - 2 are done;
             // the MMA warp read that tile's flag (same slot) before issuing them
             if (gg >= 2 && !waitb(p, ms, &ms.pv_done[gg & 1], ((gg - 2) >> 1) & 1)) return;
@@ -851,8 +857,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     for (int e = 0; e < 8; ++e) row[e] = make_uint4(0, 0, 0, 0);
                 }
             }
-            // a flagged warp's weights are rewritten below, and its sums added then
-            store_p(s, kvs, !wex, gg);
+            put_p(hw, lw, gg);
             if (lane == 0) ptx::mbar_arrive(&ms.p_full[gg & 1]);
 
             // every warp has written its weights and its flag for tile gg
@@ -908,7 +913,8 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                     }
                 }
             }
-            store_p(s, kvs, wex, gg);
+            make_p(s, kvs, wex, hw, lw);
+            put_p(hw, lw, gg);
             if (lane == 0) ptx::mbar_arrive(&ms.p_redo);
         }
         g = g0 + nt;
@@ -1043,7 +1049,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(&ms.q_ready, kSoftmaxWarps);
         ptx::mbar_init(&ms.q_full, 1);
         ptx::mbar_init(&ms.o_free, kSoftmaxWarps);
-        ptx::mbar_init(&ms.drain, 1);
+        ptx::mbar_init(&ms.drain, 2);       // one commit per MMA issuer
         ptx::mbar_init(&ms.all_sync, kSoftmaxWarps);
         ptx::mbar_init(&ms.p_redo, kSoftmaxWarps);
         ms.redo[0] = ms.redo[1] = 0;
@@ -1065,7 +1071,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0)
         producer<kFp8>(p, &map_a, &map_b, smem, ms, slot);
     else if (warp == 1)
-        mma_issuer<kFp8>(p, smem, ms, slot);
+        score_issuer<kFp8>(p, smem, ms, slot);
+    else if (warp == kValueWarp)
+        value_issuer<kFp8>(p, smem, ms, slot);
     else
         softmax_role<kFp8>(p, smem, ms, slot, g_idx, &map_out, &map_part);
 
