@@ -95,18 +95,28 @@ struct Cfg {
     // KV stage.  The MMAs read the tile as 128-byte-wide column chunks (FP8: 4
     // chunks of 128 latent dims; bf16: 9 chunks of 64 dims, the last one the
     // RoPE part) of 128 positions, each chunk a stack of 8-position x 128 B
-    // swizzle atoms.  Byte offset of (8-position group g, chunk c):
-    //   g * kGroupStride + c * kChunkStride
-    // FP8: one 8 KB box per page lands [half][chunk][8 rows][128 B], so the
-    //   group stride is 4 KB and the chunks are 1 KB apart; the RoPE part is a
-    //   separate [128 positions][64 B] region at kRopeOff.
+    // swizzle atoms.  The c_kv chunks are copied and freed in parts of kCpp
+    // chunks (FP8: one part; parts of one or two chunks, which free each
+    // chunk as soon as its value MMAs are done, measured slower: the smaller
+    // copies cost more than the earlier start gains).  Byte offset of
+    // (8-position group g, chunk c):
+    //   g * kGroupStride + chunk_off(c)
+    // FP8: part h holds chunks [h kCpp, (h+1) kCpp) in a region of its own; one
+    //   box per (page, part) lands [half][chunk][8 rows][128 B] there, so the
+    //   group stride is kCpp KB and the part's chunks are 1 KB apart; the RoPE
+    //   part is a separate [128 positions][64 B] region at kRopeOff.
     // bf16: one 2 KB box per (page, chunk): chunks of [128 positions][128 B].
     static constexpr int kDimChunks = kFp8 ? 4 : 8;                               // 128-B chunks of c_kv
-    static constexpr int kGroupStride = kFp8 ? 4096 : 1024;
-    static constexpr int kChunkStride = kFp8 ? 1024 : kTileM * 128;
+    static constexpr int kCpp = kFp8 ? 4 : 1;                                     // chunks per c_kv part
+    static constexpr int kGroupStride = kFp8 ? kCpp * 1024 : 1024;
+    static constexpr int kChunkStride = kFp8 ? 1024 : kTileM * 128;               // within a part
+    static constexpr int kPartStride = kTileM * kCpp * 128;                       // c_kv part regions
+    __host__ __device__ static constexpr int chunk_off(int c) {
+        return (c / kCpp) * kPartStride + (c % kCpp) * kChunkStride;
+    }
     static constexpr int kRopeOff = kFp8 ? 4 * 16384 : 8 * kTileM * 128;
     static constexpr int kStageBytes = kFp8 ? 4 * 16384 + kTileM * 64 : 9 * kTileM * 128;
-    static constexpr int kVChunks = kFp8 ? 1 : 8;                                 // parts holding c_kv
+    static constexpr int kVChunks = kDimChunks / kCpp;                            // parts holding c_kv
     static constexpr int kKvOff = 0;
     static constexpr int kScaleOff = kKvOff + kStages * kStageBytes;               // FP8: 512 B / stage
     static constexpr int kScaleBytes = kFp8 ? kTileM * 4 : 0;
@@ -127,7 +137,7 @@ struct Cfg {
     static constexpr int kParts = kVChunks + 1;
     static constexpr int kRope = kVChunks;                                        // part index of the RoPE chunk
     __host__ __device__ static constexpr uint32_t part_bytes(int part) {            // per page
-        return kFp8 ? (part == kRope ? 1024u : 8192u + 64u) : 2048u;
+        return kFp8 ? (part == kRope ? 1024u : 2048u * kCpp + (part == 0 ? 64u : 0u)) : 2048u;
     }
     // exponent offset C and lazy threshold TAU of the softmax stabiliser, and
     // the headroom DELTA it is placed above a new maximum when it moves (so
@@ -282,9 +292,10 @@ __device__ void producer(const Problem &p, const CUtensorMap *map_a, const CUten
                     if (part == C::kRope) {
                         ptx::tma_load_2d_hint(st + C::kRopeOff + lane * 1024, map_b, bar, 512, y, pol);
                     } else {
-                        // page slot `lane` = 8-position groups 2*lane, 2*lane+1
-                        ptx::tma_load_5d_hint(st + lane * 2 * C::kGroupStride, map_a, bar, 0, 0, 0, 0, pid, pol);
-                        if (!p.kv_scale_per_tensor)
+                        // page slot `lane` = 8-position groups 2*lane, 2*lane+1 of the part
+                        ptx::tma_load_5d_hint(st + part * C::kPartStride + lane * 2 * C::kGroupStride, map_a, bar, 0,
+                                              0, part * C::kCpp, 0, pid, pol);
+                        if (part == 0 && !p.kv_scale_per_tensor)
                             ptx::bulk_load_hint(smem + C::kScaleOff + stage * C::kScaleBytes + lane * 64,
                                                 p.kv_scale + (int64_t)pid * kPage, 64, bar, pol);
                     }
@@ -373,12 +384,12 @@ __device__ void score_issuer(const Problem &p, unsigned char *smem, Misc &ms, in
                     ptx::mma_f8(d, dr_kv + so + 2 * ks, dr_q + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
             } else {
 #pragma unroll
-                for (int c = 0; c < C::kDimChunks; ++c) {
-                    const uint64_t a = dq_kv + so + c * (C::kChunkStride >> 4);
+                for (int c = part * C::kCpp; c < (part + 1) * C::kCpp; ++c) {
+                    const uint64_t a = dq_kv + so + (C::chunk_off(c) >> 4);
                     const uint64_t b = dq_q + c * (C::kQChunk >> 4);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        ptx::mma_f8(d, a + 2 * ks, b + 2 * ks, idesc_qk, (first && c == 0 && ks == 0) ? 0u : 1u);
+                        ptx::mma_f8(d, a + 2 * ks, b + 2 * ks, idesc_qk, (first && ks == 0) ? 0u : 1u);
                 }
             }
         } else {
@@ -444,8 +455,9 @@ __device__ void value_issuer(const Problem &p, unsigned char *smem, Misc &ms, in
             if constexpr (kFp8) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)  // 32 positions (4 groups) per MMA; N = 96: P hi | P lo
-                    ptx::mma_f8(d, a0 + m * (C::kChunkStride >> 4) + ks * ((4 * C::kGroupStride) >> 4),
+                    ptx::mma_f8(d, a0 + (C::chunk_off(m) >> 4) + ks * ((4 * C::kGroupStride) >> 4),
                                 pb + ks * (512 >> 4), idesc_pv, (first && ks == 0) ? 0u : 1u);
+                if (m % C::kCpp == C::kCpp - 1) ptx::mma_commit(&ms.part_empty[stage][m / C::kCpp]);
             } else {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)  // 16 positions (2 groups) per MMA
@@ -455,7 +467,6 @@ __device__ void value_issuer(const Problem &p, unsigned char *smem, Misc &ms, in
                 ptx::mma_commit(&ms.part_empty[stage][2 * m + 1]);
             }
         }
-        if constexpr (kFp8) ptx::mma_commit(&ms.part_empty[stage][0]);
     };
 
     uint32_t g = 0, pi = 0;
@@ -841,7 +852,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             // a flagged warp's weights are rewritten below, and its sums added then
             make_p(s, kvs, !wex, hw, lw);
             // P buffer gg & 1 is free once the value MMAs of tile gg - 2 are done;
-            // the MMA warp read that tile's flag (same slot) before issuing them
+            // the value warp read that tile's flag (same slot) before issuing them
             if (gg >= 2 && !waitb(p, ms, &ms.pv_done[gg & 1], ((gg - 2) >> 1) & 1)) return;
             if (wex && lane == 0) *reinterpret_cast<volatile uint32_t *>(&ms.redo[gg & 1]) = gg + 1;
             // rows past the context, and page slots this tile did not load, may
@@ -851,7 +862,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
                 unsigned char *stg = smem + C::kKvOff + stage * C::kStageBytes;
 #pragma unroll
                 for (int c = 0; c < C::kDimChunks; ++c) {
-                    uint4 *row = reinterpret_cast<uint4 *>(stg + (i >> 3) * C::kGroupStride + c * C::kChunkStride +
+                    uint4 *row = reinterpret_cast<uint4 *>(stg + (i >> 3) * C::kGroupStride + C::chunk_off(c) +
                                                            (i & 7) * 128);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) row[e] = make_uint4(0, 0, 0, 0);
@@ -960,38 +971,47 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
             // ln sum_j exp(score_j) = (m2c + log2 l) * ln 2
             row_lse = (bad_rows >> hst) & 1u ? NAN : (l > 0.f ? (ms.m2c[cb + hst] + __log2f(l)) * kLn2 : -INFINITY);
         }
-        // O goes out one 128-dim block at a time, each row group on its own:
-        // the group's threads write their dims of its 16 rows into a [16][128]
-        // staging box (two per group alternate, in the query area, free until
-        // the next piece), and the group's first thread stores the box with a
-        // tensor store; the maps clip rows past the sequence's R.
+        // O goes out in 128-dim blocks, each row group on its own: the group's
+        // threads write their dims of its 16 rows into [16][128] staging boxes
+        // (in the query area, free until the next piece: 16 KB per group, so
+        // all four blocks at once for bf16 boxes, two at a time for fp32),
+        // and the group's first thread stores them with tensor stores; the
+        // maps clip rows past the sequence's R.
         const int nrows = min(kRpt, rows_here - cb);
         const bool f32_box = pc.single && p.out_f32;   // partials are bf16
-        constexpr int kBoxBytes = kRpt * 128 * 4;
+        const int per_round = f32_box ? 2 : 4;
+        const int box_bytes = kRpt * 128 * (f32_box ? 4 : 2);
+        unsigned char *boxes = smem + C::kQOff + h * (4 * kRpt * 128 * 2);
 #pragma unroll 1
-        for (int m = 0; m < 4; ++m) {
-            unsigned char *box = smem + C::kQOff + (2 * h + (m & 1)) * kBoxBytes;
-            if (m >= 2) {  // the store of block m - 2 has finished reading this box
-                if (hst == 0) ptx::bulk_wait_read<1>();
+        for (int m0 = 0; m0 < 4; m0 += per_round) {
+            if (m0 > 0) {  // the previous round's stores have finished reading the boxes
+                if (hst == 0) ptx::bulk_wait_read<0>();
                 if (!hsync(p, ms)) return;
             }
-            float o[kRpt];
-            tmem_rows<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
+#pragma unroll 1
+            for (int m = m0; m < m0 + per_round; ++m) {
+                unsigned char *box = boxes + (m - m0) * box_bytes;
+                float o[kRpt];
+                tmem_rows<kFp8>(tmem + C::kColO + C::kOStride * m + cb, o);
 #pragma unroll
-            for (int c = 0; c < kRpt; ++c) {
-                const float v = o[c] * inv_l[c];
-                if (f32_box)
-                    reinterpret_cast<float *>(box)[c * 128 + i] = v;
-                else
-                    reinterpret_cast<__nv_bfloat16 *>(box)[c * 128 + i] = __float2bfloat16_rn(v);
+                for (int c = 0; c < kRpt; ++c) {
+                    const float v = o[c] * inv_l[c];
+                    if (f32_box)
+                        reinterpret_cast<float *>(box)[c * 128 + i] = v;
+                    else
+                        reinterpret_cast<__nv_bfloat16 *>(box)[c * 128 + i] = __float2bfloat16_rn(v);
+                }
             }
             ptx::fence_proxy_async_smem();
             if (!hsync(p, ms)) return;
             if (hst == 0 && nrows > 0) {
-                if (pc.single)
-                    ptx::tma_store_3d(map_out, box, 128 * m, r0 + cb, pc.b);
-                else
-                    ptx::tma_store_3d(map_part, box, 128 * m, (int)pc.piece, r0 + cb);
+                for (int m = m0; m < m0 + per_round; ++m) {
+                    unsigned char *box = boxes + (m - m0) * box_bytes;
+                    if (pc.single)
+                        ptx::tma_store_3d(map_out, box, 128 * m, r0 + cb, pc.b);
+                    else
+                        ptx::tma_store_3d(map_part, box, 128 * m, (int)pc.piece, r0 + cb);
+                }
                 ptx::bulk_commit();
             }
         }
@@ -1124,7 +1144,7 @@ bool make_fp8_latent_map(CUtensorMap *map, const void *base, int num_pages) {
     if (!encode) return false;
     const cuuint64_t dims[5] = {128, 8, 4, 2, (cuuint64_t)num_pages};
     const cuuint64_t strides[4] = {(cuuint64_t)kD, 128, (cuuint64_t)8 * kD, (cuuint64_t)kPage * kD};
-    const cuuint32_t box[5] = {128, 8, 4, 2, 1};
+    const cuuint32_t box[5] = {128, 8, (cuuint32_t)Cfg<true>::kCpp, 2, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1189,7 +1209,7 @@ int launch_impl(const Problem &p, cudaStream_t stream) {
 
 static_assert(smem_bytes<true>() <= 232448, "FP8 tile does not fit shared memory");
 static_assert(2 * kRowGroups * kRpt * 128 * 4 <= Cfg<true>::kQBytes && 2 * kRowGroups * kRpt * 128 * 4 <= Cfg<false>::kQBytes,
-              "each row group's two epilogue staging boxes must fit the query area");
+              "each row group's 16 KB of epilogue staging boxes must fit the query area");
 static_assert(smem_bytes<false>() <= 232448, "bf16 tile does not fit shared memory");
 static_assert(Cfg<true>::kColO + 3 * Cfg<true>::kOStride + Cfg<true>::kNMma <= kTmemCols, "TMEM overflow");
 static_assert(Cfg<false>::kColO + 3 * Cfg<false>::kOStride + Cfg<false>::kNMma <= kTmemCols, "TMEM overflow");
