@@ -110,9 +110,7 @@ __device__ __forceinline__ int total_pages(const Problem &p) {
         int np = b < p.B ? seq_pages(p, b, &bad) : 0;
         acc += np;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    return acc;
+    return (int)__reduce_add_sync(0xffffffffu, (unsigned)acc);  // one warp reduction instruction
 }
 
 // Schedule facts for b = base + lane; run_* carry the sums of earlier chunks.

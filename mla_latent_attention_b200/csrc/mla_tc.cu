@@ -210,12 +210,6 @@ __device__ __forceinline__ int ntiles_of(const Piece &pc) {
     return (pc.page_hi - pc.page_lo + kTilePages - 1) / kTilePages;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
 // Reduces 16 per-lane values x[r] + off (one per row) over the warp's 32
 // lanes by halving exchanges (8 + 4 + 2 + 1 + 1 shuffles instead of 16 x 5):
 // the result for row r is returned in lanes 2r and 2r + 1.
@@ -558,9 +552,9 @@ __device__ bool stage_query(const Problem &p, unsigned char *smem, Misc &ms, int
                 mbits = __vmaxu2(mbits, v[j][h].w & 0x7FFF7FFFu);
             }
         }
-        mbits = max(mbits & 0xFFFFu, mbits >> 16);
+        // the warp's largest magnitude bits in one reduction instruction
+        mbits = __reduce_max_sync(0xffffffffu, max(mbits & 0xFFFFu, mbits >> 16));
         float amax = __uint_as_float(mbits << 16);
-        amax = warp_max(amax);
         if ((threadIdx.x & 31) == 0) ms.amax[(threadIdx.x >> 5) - 2] = amax;
         if (!gsync(p, ms)) return false;   // also: every raw read is done
 #pragma unroll
