@@ -99,13 +99,13 @@ def _check(rc: int, what: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()   # the argtypes are c_void_p: a plain int converts
 
 
 def _stream(stream, device):
     if stream is None:
         stream = torch.cuda.current_stream(device)
-    return ctypes.c_void_p(stream.cuda_stream)
+    return stream.cuda_stream
 
 
 def _kv_code(kv_pages):
@@ -138,13 +138,14 @@ def workspace_size(dims: Dims) -> int:
 
 
 def _need(t, name, dtype=None, device=None, shape=None):
-    if t.device.type != "cuda":
+    d = t.device
+    if d.type != "cuda":
         raise MlaError(f"{name} must be a CUDA tensor")
-    if device is not None and t.device != device:
-        raise MlaError(f"{name} is on {t.device}, expected {device}")
+    if device is not None and d != device:
+        raise MlaError(f"{name} is on {d}, expected {device}")
     if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
         raise MlaError(f"{name} has dtype {t.dtype}")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise MlaError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if name != "page_table" and not t.is_contiguous():
         raise MlaError(f"{name} must be contiguous")

@@ -54,6 +54,9 @@
 // Every wait is bounded: after 4e9 SM cycles (about two seconds) the CTA
 // records a timeout in the error word, stops, drains its outstanding copies
 // and MMAs and frees its tensor memory.
+#include <atomic>
+#include <mutex>
+
 #include <cuda.h>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
@@ -1114,6 +1117,48 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
+// Encoded tensor maps are remembered by everything that defines them (the
+// map kind, base address and extents): encoding is host work of a few
+// microseconds, and a decode step asks for the same four maps per layer at
+// every step.  A map holds no reference to the memory it describes, so an
+// entry stays right for any allocation at the same address and extents.
+struct MapKey {
+    const void *base;
+    uint64_t a, b, c;
+    int kind;
+    bool operator==(const MapKey &o) const {
+        return base == o.base && a == o.a && b == o.b && c == o.c && kind == o.kind;
+    }
+};
+
+template <typename Make>
+bool cached_map(const MapKey &k, CUtensorMap *out, Make &&make) {
+    constexpr int kEntries = 256;
+    struct Entry {
+        MapKey key;
+        CUtensorMap map;
+        bool valid;
+    };
+    static Entry cache[kEntries];
+    static std::mutex mu;
+    uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+    h ^= (k.a + 31 * k.b + 961 * k.c + 29791 * (uint64_t)k.kind) * 0xC2B2AE3D27D4EB4Full;
+    Entry &e = cache[(h >> 32) % kEntries];
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (e.valid && e.key == k) {
+            *out = e.map;
+            return true;
+        }
+    }
+    if (!make(out)) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    e.key = k;
+    e.map = *out;
+    e.valid = true;
+    return true;
+}
+
 // 2-D view of the page pool: [num_pages*16 rows][576 elements], boxes of 16 rows.
 bool make_kv_map(CUtensorMap *map, const void *base, int num_pages, bool fp8, uint32_t box_cols,
                  CUtensorMapSwizzle swz) {
@@ -1179,17 +1224,42 @@ template <bool kFp8>
 int launch_impl(const Problem &p, cudaStream_t stream) {
     CUtensorMap ma, mb, mo, mp;
     bool ok;
+    const uint64_t np = (uint64_t)p.num_pages;
     if (kFp8) {
-        ok = make_fp8_latent_map(&ma, p.kv, p.num_pages) &&
-             make_kv_map(&mb, p.kv, p.num_pages, true, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+        ok = cached_map({p.kv, np, 0, 0, 0}, &ma, [&](CUtensorMap *m) { return make_fp8_latent_map(m, p.kv, p.num_pages); }) &&
+             cached_map({p.kv, np, 0, 0, 1}, &mb, [&](CUtensorMap *m) {
+                 return make_kv_map(m, p.kv, p.num_pages, true, 64, CU_TENSOR_MAP_SWIZZLE_64B);
+             });
     } else {
-        ok = make_kv_map(&ma, p.kv, p.num_pages, false, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = cached_map({p.kv, np, 0, 0, 2}, &ma, [&](CUtensorMap *m) {
+            return make_kv_map(m, p.kv, p.num_pages, false, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+        });
         mb = ma;
     }
-    ok = ok && make_out_maps(&mo, &mp, p);
+    // (make_out_maps encodes both output maps; each cached entry keeps one)
+    ok = ok && cached_map({p.out, (uint64_t)p.R, (uint64_t)p.B, (uint64_t)p.out_f32, 3}, &mo, [&](CUtensorMap *m) {
+             CUtensorMap unused;
+             return make_out_maps(m, &unused, p);
+         });
+    if (ok && (p.max_pieces < 1 || !p.part_o)) {
+        mp = mo;  // no partials: never stored through
+    } else if (ok) {
+        ok = cached_map({p.part_o, (uint64_t)p.max_pieces, (uint64_t)p.R, 0, 4}, &mp, [&](CUtensorMap *m) {
+            CUtensorMap unused;
+            return make_out_maps(&unused, m, p);
+        });
+    }
     if (!ok) return MLA_ERR_CUDA;
     const int smem = smem_bytes<kFp8>();
-    cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the shared-memory attribute is set once per device
+    static std::atomic<uint64_t> attr_set{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    const uint64_t bit = dev < 64 ? 1ull << dev : 0;
+    if (e == cudaSuccess && (!bit || !(attr_set.load() & bit))) {
+        e = cudaFuncSetAttribute(tc_decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess && bit) attr_set.fetch_or(bit);
+    }
     if (e == cudaSuccess) {
         tc_decode_kernel<kFp8><<<p.n_slots * p.n_groups, kThreads, smem, stream>>>(p, ma, mb, mo, mp);
         e = cudaGetLastError();
