@@ -175,9 +175,16 @@ def test_reference_arm_under_torchrun_two_ranks():
 
 
 def test_split_step_divides_the_timed_layer():
-    """The per-kernel times are the timed per-layer time divided in the
-    proportion the event nodes measured, so they add up to the step."""
-    att, mer = bench.split_step(60.0, 66.0, 11.0)
-    assert abs(att + mer - 60.0) < 1e-9
-    assert abs(att / mer - 6.0) < 1e-9
+    """The event nodes' own latency (half the amount by which the two
+    event-measured times exceed the timed layer) comes off each kernel, so
+    the two add up to the step."""
+    att, mer = bench.split_step(54.69, 56.75, 10.23)
+    assert abs(att + mer - 54.69) < 1e-9
+    assert abs(mer - (10.23 - (56.75 + 10.23 - 54.69) / 2)) < 1e-9
+    # event times that do not exceed the step: nothing is taken off
+    att, mer = bench.split_step(60.0, 50.0, 10.0)
+    assert (att, mer) == (50.0, 10.0)
+    # a merge shorter than the event latency counts as zero
+    att, mer = bench.split_step(10.0, 30.0, 1.0)
+    assert (att, mer) == (10.0, 0.0)
     assert bench.split_step(10.0, 0.0, 0.0) == (10.0, 0.0)
