@@ -472,9 +472,9 @@ def split_step(layer_us, att_ev, mer_ev):
     kernel of the event-instrumented copy sits between two event nodes, which
     add the same latency to each: that latency is half the amount by which
     the two event-measured times exceed the timed layer, and it is taken off
-    both.  (On the 142K layer this puts the merge at 4.1 us, as a copy of the
-    library without the merge measured on the same box, where a split in
-    proportion to the event times gave it 8.4 us.)"""
+    both.  (On the 142K layer this puts the merge at 4.4 us of the layer; the
+    step timed with and without the merge on one GPU differs by 4.1 us, where
+    a split in proportion to the event times gave the merge 8.4 us.)"""
     if att_ev + mer_ev <= 0:
         return layer_us, 0.0
     extra = max(0.0, (att_ev + mer_ev - layer_us) / 2.0)

@@ -981,7 +981,7 @@ __device__ void softmax_role(const Problem &p, unsigned char *smem, Misc &ms, in
         unsigned char *boxes = smem + C::kQOff + h * (4 * kRpt * 128 * 2);
 #pragma unroll 1
         for (int m0 = 0; m0 < 4; m0 += per_round) {
-            if (m0 > 0) {  // the previous round's stores have finished reading the boxes
+            if (m0 > 0) {  // the stores of the previous blocks have finished reading the boxes
                 if (hst == 0) ptx::bulk_wait_read<0>();
                 if (!hsync(p, ms)) return;
             }
