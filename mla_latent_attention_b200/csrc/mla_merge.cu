@@ -170,14 +170,33 @@ __device__ __forceinline__ void merge_unit_warp(const T *o0, int64_t o_stride, c
 template <bool kCta>
 __global__ void __launch_bounds__(kThreads, kCta ? 3 : 1) merge_internal_kernel(Problem p) {
     __shared__ MergeSmem sm;
-    const int64_t unit = kCta ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    __shared__ int row_info[kWarps / kQuarters][2];  // warp per unit: pieces of the CTA's rows
+    const int warp = threadIdx.x >> 5;
+    const int64_t unit = kCta ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kWarps + warp;
     const int64_t grow = unit / kQuarters;  // b * R + r
-    if (grow >= (int64_t)p.B * p.R) return;
+    const bool valid = grow < (int64_t)p.B * p.R;
     const int quarter = (int)(unit % kQuarters);
-    const int b = (int)(grow / p.R), r = (int)(grow % p.R);
+    const int b = valid ? (int)(grow / p.R) : 0, r = valid ? (int)(grow % p.R) : 0;
     int n_pieces = 0, piece_base = 0;
     bool bad = false;
-    pieces_of(p, b, &n_pieces, &piece_base, &bad);
+    if (kCta) {
+        if (!valid) return;
+        pieces_of(p, b, &n_pieces, &piece_base, &bad);
+    } else {
+        // the CTA's warps cover kWarps / kQuarters rows, four warps each: the
+        // first warp of each row scans the schedule for the row's sequence
+        if (warp % kQuarters == 0) {
+            if (valid) pieces_of(p, b, &n_pieces, &piece_base, &bad);
+            if ((threadIdx.x & 31) == 0) {
+                row_info[warp / kQuarters][0] = n_pieces;
+                row_info[warp / kQuarters][1] = piece_base;
+            }
+        }
+        __syncthreads();
+        if (!valid) return;
+        n_pieces = row_info[warp / kQuarters][0];
+        piece_base = row_info[warp / kQuarters][1];
+    }
     if (n_pieces < 2) return;  // finished by the decode kernel
     // The kernel may start while the attention kernel is finishing (its
     // schedule needs only ctx_lens); the partials are read after it is done.
