@@ -183,7 +183,17 @@ __global__ void __launch_bounds__(kThreads, kCta ? 3 : 4) merge_internal_kernel(
     bool bad = false;
     if (kCta) {
         if (!valid) return;
-        pieces_of(p, b, &n_pieces, &piece_base, &bad);
+        // one warp scans the schedule for the CTA's row
+        if (warp == 0) {
+            pieces_of(p, b, &n_pieces, &piece_base, &bad);
+            if ((threadIdx.x & 31) == 0) {
+                row_info[0][0] = n_pieces;
+                row_info[0][1] = piece_base;
+            }
+        }
+        __syncthreads();
+        n_pieces = row_info[0][0];
+        piece_base = row_info[0][1];
     } else {
         // the CTA's warps cover kWarps / kQuarters rows, four warps each: the
         // first warp of each row scans the schedule for the row's sequence
