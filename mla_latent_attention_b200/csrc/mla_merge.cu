@@ -247,7 +247,10 @@ int launch_merge_internal(const Problem &p, cudaStream_t stream) {
     if (rows <= 0) return MLA_OK;
     // Slots much more numerous than sequences mean many pieces per sequence:
     // eight warps per unit.  Otherwise a warp per unit (it handles any number
-    // of pieces, only more slowly when there are many).
+    // of pieces, only more slowly when there are many).  The choice depends on
+    // the schedule alone, not on the row count, so that padding the heads of
+    // a call changes none of its results: the two forms combine the parts in
+    // different orders.
     const bool many = p.n_slots > 2 * p.B;
     const int64_t units = rows * kQuarters;
     // a programmatic dependent of the attention kernel before it in the stream

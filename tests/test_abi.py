@@ -44,6 +44,20 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(mla.EXPORTED) <= exported
 
 
+def test_library_leaves_none_of_its_own_symbols_undefined():
+    """A shared library links even with references it does not define; they
+    only fail when first called.  Every function of the library's namespace
+    must be defined in the library itself."""
+    import shutil
+    import subprocess
+    if not shutil.which("nm"):
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--undefined-only", mla.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    missing = [ln.split()[-1] for ln in out.splitlines() if "3mla" in ln or " mla_" in ln]
+    assert not missing, missing
+
+
 def test_library_is_sm100a_only():
     """The fatbinary is built for sm_100a (checked on the build command, not the binary)."""
     assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
